@@ -1,0 +1,100 @@
+"""Seeded synthetic inputs for the KDA operator.
+
+This module draws random numbers and nothing else: it holds none of the
+operator's arithmetic, so the tests, the benchmark and the fp64 oracle can all
+take their inputs from it.  Everything is drawn on the CPU with a seeded
+``torch.Generator`` and returned as CPU tensors.
+
+Distributions (the workloads of the KDA operator description):
+  q, k ~ N(0, 1), then L2-normalised per (token, head) over the key channels;
+  v ~ N(0, 1);  g ~ N(0, 1) per key channel (the raw gate: the operator applies
+  log a = -5 * sigmoid(g) itself);  beta = sigmoid(N(0, 1)) per (token, head);
+  h0 ~ N(0, std^2) in fp32 when a carried state is requested.
+Values are drawn in fp32 and rounded to the requested dtype (bf16 rounding is
+round-to-nearest-even); states stay fp32.
+"""
+from dataclasses import dataclass
+from typing import List, Optional
+
+import torch
+
+
+@dataclass
+class PrefillInputs:
+    q: torch.Tensor            # [T_tot, H, dk]
+    k: torch.Tensor            # [T_tot, H, dk]
+    v: torch.Tensor            # [T_tot, H, dv]
+    g: torch.Tensor            # [T_tot, H, dk]
+    beta: torch.Tensor         # [T_tot, H]
+    h0: Optional[torch.Tensor]  # [N, H, dk, dv] fp32 or None
+    cu_seqlens: torch.Tensor   # [N+1] int32
+
+    @property
+    def lengths(self) -> List[int]:
+        cu = self.cu_seqlens.tolist()
+        return [cu[i + 1] - cu[i] for i in range(len(cu) - 1)]
+
+
+def _unit_rows(x: torch.Tensor) -> torch.Tensor:
+    n = x.norm(dim=-1, keepdim=True)
+    return x / torch.where(n > 0, n, torch.ones_like(n))
+
+
+def cu_from_lengths(lengths) -> torch.Tensor:
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + int(L))
+    return torch.tensor(cu, dtype=torch.int32)
+
+
+def make_prefill(lengths, H: int, dk: int, dv: int, dtype=torch.bfloat16,
+                 seed: int = 0, h0_std: Optional[float] = None
+                 ) -> PrefillInputs:
+    """Packed varlen prefill inputs for sequences of the given lengths."""
+    gen = torch.Generator().manual_seed(int(seed))
+    T = int(sum(lengths))
+    N = len(lengths)
+    q = _unit_rows(torch.randn(T, H, dk, generator=gen))
+    k = _unit_rows(torch.randn(T, H, dk, generator=gen))
+    v = torch.randn(T, H, dv, generator=gen)
+    g = torch.randn(T, H, dk, generator=gen)
+    beta = torch.sigmoid(torch.randn(T, H, generator=gen))
+    h0 = None
+    if h0_std is not None:
+        h0 = torch.randn(N, H, dk, dv, generator=gen) * float(h0_std)
+    return PrefillInputs(q.to(dtype), k.to(dtype), v.to(dtype), g.to(dtype),
+                         beta.to(dtype), h0, cu_from_lengths(lengths))
+
+
+def draw_lengths(n: int, lo: int, hi: int, seed: int) -> List[int]:
+    """n integer lengths uniform on [lo, hi] (both ends inclusive)."""
+    gen = torch.Generator().manual_seed(int(seed))
+    return torch.randint(lo, hi + 1, (n,), generator=gen).tolist()
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor     # [B, H, dk]
+    k: torch.Tensor     # [B, H, dk]
+    v: torch.Tensor     # [B, H, dv]
+    g: torch.Tensor     # [B, H, dk]
+    beta: torch.Tensor  # [B, H]
+
+
+def make_decode_step(B: int, H: int, dk: int, dv: int, dtype=torch.bfloat16,
+                     seed: int = 0) -> DecodeInputs:
+    """One token per (sequence, head) with the prefill distributions."""
+    gen = torch.Generator().manual_seed(int(seed))
+    q = _unit_rows(torch.randn(B, H, dk, generator=gen))
+    k = _unit_rows(torch.randn(B, H, dk, generator=gen))
+    v = torch.randn(B, H, dv, generator=gen)
+    g = torch.randn(B, H, dk, generator=gen)
+    beta = torch.sigmoid(torch.randn(B, H, generator=gen))
+    return DecodeInputs(q.to(dtype), k.to(dtype), v.to(dtype), g.to(dtype),
+                        beta.to(dtype))
+
+
+def make_state(B: int, H: int, dk: int, dv: int, std: float, seed: int
+               ) -> torch.Tensor:
+    gen = torch.Generator().manual_seed(int(seed))
+    return torch.randn(B, H, dk, dv, generator=gen) * float(std)

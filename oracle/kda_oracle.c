@@ -1,0 +1,164 @@
+/*
+ * kda_oracle.c -- fp64 CPU oracle for the Kimi Delta Attention (KDA) recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct
+ * definition that the CUDA path of libkda is checked against.  Only tests/,
+ * __graft_entry__.smoke() and bench.py's CPU-baseline leg may load it.  It
+ * shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (one head of one sequence, token by token, in fp64):
+ *
+ *   log a_t = -5 * sigmoid(g_t)                      per key channel
+ *   S       = Diag(a_t) S                            decay the old state first
+ *   u_t     = beta_t * (v_t - S^T k_t)               delta-rule error, read with
+ *                                                    the *decayed* state
+ *   S       = S + k_t u_t^T                          write only the difference
+ *   o_t     = S^T q_t                                read from the *updated* state
+ *
+ * Sources (web pages on Kimi K3):
+ *   - "Kimi K3 发布核实与 Moonshot AI 主干架构演变" (dllmharness report), §3,
+ *     paragraph "KDA 为什么不同于 MLA": per-head state matrix; per-channel
+ *     retention alpha decays the old state first, then the write strength beta
+ *     with the current key and value corrects it, and the query reads the
+ *     updated state.
+ *   - same page, §3, "K3 对 Kimi Linear 的进一步修改", bullet 1: the
+ *     log-decay is a scaled sigmoid bounded below by -5.
+ *   - "Kimi K3 模型架构解析：KDA、AttnRes 与 Stable LatentMoE", §二.2
+ *     (S_t = Update(S_{t-1}, k_t, v_t), o_t = Read(S_t, q_t)) and §二.3
+ *     (delta rule: read the old mapping with the key, take the error
+ *     against the value, write back only the difference).
+ *
+ * Readings where the pages are silent: beta arrives already in (0,1); no
+ * query scale; q and k are used as given (their normalisation belongs to the
+ * input); sequences restart from h0 (or zero) at each cu_seqlens boundary.
+ *
+ * Layouts (row-major, last index contiguous), all fp64:
+ *   q, k, g  [T_tot, H, dk]      v, o  [T_tot, H, dv]      beta [T_tot, H]
+ *   h0, hT   [N, H, dk, dv]      cu_seqlens int64 [N+1]
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* log a = -5 * sigmoid(g), written so that g = +/-inf give exact limits. */
+static double log_alpha(double g)
+{
+    double s;
+    if (g >= 0.0) {
+        s = 1.0 / (1.0 + exp(-g));
+    } else {
+        double e = exp(g);
+        s = e / (1.0 + e);
+    }
+    return -5.0 * s;
+}
+
+/* One token of the recurrence on one head's state S [dk][dv] (in place).
+ * o may be NULL.  r is scratch of length dv. */
+static void kda_token(double *S, int dk, int dv,
+                      const double *q, const double *k, const double *v,
+                      const double *g, double beta, double *o, double *r)
+{
+    /* decay first */
+    for (int i = 0; i < dk; ++i) {
+        double a = exp(log_alpha(g[i]));
+        double *row = S + (size_t)i * dv;
+        for (int j = 0; j < dv; ++j) row[j] *= a;
+    }
+    /* r = S^T k with the decayed state */
+    for (int j = 0; j < dv; ++j) r[j] = 0.0;
+    for (int i = 0; i < dk; ++i) {
+        const double *row = S + (size_t)i * dv;
+        double ki = k[i];
+        for (int j = 0; j < dv; ++j) r[j] += row[j] * ki;
+    }
+    /* u = beta (v - r);  S += k u^T */
+    for (int j = 0; j < dv; ++j) r[j] = beta * (v[j] - r[j]);
+    for (int i = 0; i < dk; ++i) {
+        double *row = S + (size_t)i * dv;
+        double ki = k[i];
+        for (int j = 0; j < dv; ++j) row[j] += ki * r[j];
+    }
+    /* o = S^T q with the updated state */
+    if (o) {
+        for (int j = 0; j < dv; ++j) o[j] = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            const double *row = S + (size_t)i * dv;
+            double qi = q[i];
+            for (int j = 0; j < dv; ++j) o[j] += row[j] * qi;
+        }
+    }
+}
+
+/*
+ * Prefill: every token of every (sequence n, head h) unit whose mask byte is
+ * nonzero (mask may be NULL = all units).  Units are independent; OpenMP runs
+ * them in parallel, the tokens of a unit run in order.
+ * Returns 0, or -1 on a malformed cu_seqlens or allocation failure.
+ */
+int kda_oracle_forward(const double *q, const double *k, const double *v,
+                       const double *g, const double *beta, const double *h0,
+                       const int64_t *cu_seqlens, int N, int64_t T_tot,
+                       int H, int dk, int dv, const uint8_t *unit_mask,
+                       double *o, double *hT)
+{
+    if (cu_seqlens[0] != 0 || cu_seqlens[N] != T_tot) return -1;
+    for (int n = 0; n < N; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    int err = 0;
+    long units = (long)N * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long u = 0; u < units; ++u) {
+        if (unit_mask && !unit_mask[u]) continue;
+        int n = (int)(u / H), h = (int)(u % H);
+        double *S = (double *)malloc(sizeof(double) * ((size_t)dk * dv + dv));
+        if (!S) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        double *r = S + (size_t)dk * dv;
+        const size_t sz = (size_t)dk * dv;
+        if (h0) memcpy(S, h0 + (size_t)u * sz, sizeof(double) * sz);
+        else memset(S, 0, sizeof(double) * sz);
+        for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
+            size_t th = (size_t)t * H + h;
+            kda_token(S, dk, dv, q + th * dk, k + th * dk, v + th * dv,
+                      g + th * dk, beta[th], o ? o + th * dv : NULL, r);
+        }
+        if (hT) memcpy(hT + (size_t)u * sz, S, sizeof(double) * sz);
+        free(S);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * Decode: one token per (b, h); S [B, H, dk, dv] is updated in place and
+ * o [B, H, dv] receives the read from the updated state.  The body is the
+ * same token step as the prefill.
+ */
+int kda_oracle_decode(const double *q, const double *k, const double *v,
+                      const double *g, const double *beta, double *S,
+                      int B, int H, int dk, int dv, double *o)
+{
+    int err = 0;
+    long units = (long)B * H;
+#pragma omp parallel for schedule(static)
+    for (long u = 0; u < units; ++u) {
+        double *r = (double *)malloc(sizeof(double) * dv);
+        if (!r) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        kda_token(S + (size_t)u * dk * dv, dk, dv, q + (size_t)u * dk,
+                  k + (size_t)u * dk, v + (size_t)u * dv, g + (size_t)u * dk,
+                  beta[u], o ? o + (size_t)u * dv : NULL, r);
+        free(r);
+    }
+    return err ? -1 : 0;
+}
+
+/* The gate on its own, so tests can pin it against closed forms. */
+double kda_oracle_log_alpha(double g) { return log_alpha(g); }
