@@ -1,0 +1,196 @@
+"""Thin ctypes binding of libkda (include/kda.h).
+
+Argument marshalling only: every function here checks tensor placement,
+dtype, shape and contiguity, passes raw device pointers and the current CUDA
+stream to the C ABI, and turns a non-OK status into an exception.  All of the
+operator's arithmetic runs in libkda's CUDA kernels; there is no fallback of
+any kind, and importing a function from here on a machine without the built
+library raises immediately.
+
+The Python names are the C names.
+"""
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARGUMENT = 1
+KDA_ERR_UNSUPPORTED = 2
+KDA_ERR_WORKSPACE = 3
+KDA_ERR_CUDA = 4
+KDA_ERR_TIMEOUT = 5
+KDA_ERR_BAD_SEQLENS = 6
+
+KDA_BF16 = 0
+KDA_FP32 = 1
+
+_DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_FP32}
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, kda_status_string(status),
+                                                 status))
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libkda.so (built in-tree by gated_delta_rule_60_b200/build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(
+            "libkda.so is not built at %s; run `python -m "
+            "gated_delta_rule_60_b200.build` (nvcc, sm_100a)" % path)
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lib.kda_chunk_fwd_workspace_size.restype = sz
+    lib.kda_chunk_fwd_workspace_size.argtypes = [i32, i64, i32, i32, i32, ctypes.c_int]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                  i32, ctypes.c_int, vp, vp, vp, sz, vp]
+    lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                    i32, ctypes.c_int, vp]
+    lib.kda_stream_status.restype = ctypes.c_int
+    lib.kda_stream_status.argtypes = [vp]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_version.restype = i32
+    lib.kda_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def kda_status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> int:
+    return int(load_library().kda_version())
+
+
+def kda_chunk_fwd_workspace_size(N: int, T_tot: int, H: int, dk: int, dv: int,
+                                 dtype: torch.dtype) -> int:
+    return int(load_library().kda_chunk_fwd_workspace_size(
+        int(N), int(T_tot), int(H), int(dk), int(dv), _DTYPES[dtype]))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, shape, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device.type != "cuda" or (device is not None and t.device != device):
+        raise ValueError("%s must be on %s, got %s" % (name, device or "cuda", t.device))
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape),
+                                                            tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                  g: torch.Tensor, beta: torch.Tensor,
+                  h0: Optional[torch.Tensor] = None,
+                  cu_seqlens: Optional[torch.Tensor] = None, *,
+                  num_seqs: Optional[int] = None,
+                  o: Optional[torch.Tensor] = None,
+                  hT: Optional[torch.Tensor] = None,
+                  output_final_state: bool = True,
+                  workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked KDA prefill.  Returns (o [T_tot,H,dv], hT [N,H,dk,dv] or None).
+
+    q, k, g [T_tot, H, dk]; v [T_tot, H, dv]; beta [T_tot, H] share one dtype
+    (bf16 or fp32); h0 fp32 [N, H, dk, dv] or None; cu_seqlens int32 [N+1] on
+    the device, or None with num_seqs equal-length sequences (default 1).
+    """
+    lib = load_library()
+    dev = q.device
+    T_tot, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name, shp in ((q, "q", (T_tot, H, dk)), (k, "k", (T_tot, H, dk)),
+                         (g, "g", (T_tot, H, dk)), (v, "v", (T_tot, H, dv)),
+                         (beta, "beta", (T_tot, H))):
+        _check(t, name, dt, shp, dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty(T_tot, H, dv, dtype=dt, device=dev)
+    _check(o, "o", dt, (T_tot, H, dv), dev)
+    if hT is None and output_final_state:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    ws_need = kda_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dt)
+    if ws_need and workspace is None:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                           _ptr(h0), _ptr(cu_seqlens), N, T_tot, H, dk, dv,
+                           _DTYPES[dt], _ptr(o), _ptr(hT), _ptr(workspace),
+                           ws_bytes, _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd")
+    return o, hT
+
+
+def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    g: torch.Tensor, beta: torch.Tensor, S: torch.Tensor, *,
+                    o: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """One KDA decode step; S [B,H,dk,dv] fp32 is updated in place.
+    Returns o [B, H, dv] (dtype of q)."""
+    lib = load_library()
+    dev = q.device
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    for t, name, shp in ((q, "q", (B, H, dk)), (k, "k", (B, H, dk)),
+                         (g, "g", (B, H, dk)), (v, "v", (B, H, dv)),
+                         (beta, "beta", (B, H))):
+        _check(t, name, dt, shp, dev)
+    _check(S, "S", torch.float32, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=dt, device=dev)
+    _check(o, "o", dt, (B, H, dv), dev)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                             _ptr(S), _ptr(o), B, H, dk, dv, _DTYPES[dt],
+                             _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step")
+    return o
+
+
+def kda_stream_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(load_library().kda_stream_status(_stream_handle(stream)))

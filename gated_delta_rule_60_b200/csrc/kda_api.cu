@@ -1,0 +1,174 @@
+// kda_api.cu -- the C ABI of libkda: argument checks, dispatch, launches.
+//
+// One translation unit holds every kernel so that the per-device status word
+// (kda_common.cuh) is a single symbol.  See include/kda.h for the contract of
+// each entry point.
+#include "../../include/kda.h"
+
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+#include "kda_chunk_simt.cuh"
+#include "kda_chunk_sm100.cuh"
+
+#include <cuda_runtime.h>
+
+namespace {
+
+inline bool aligned16(const void *p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+inline bool supported_simt_d(int d) {
+    return d == 16 || d == 32 || d == 64 || d == 128;
+}
+
+template <typename T, int D>
+kda_status launch_simt(const void *q, const void *k, const void *v,
+                       const void *g, const void *beta, const float *h0,
+                       const int32_t *cu, int N, int64_t T_tot, int H,
+                       void *o, float *hT, cudaStream_t s) {
+    const size_t smem = sizeof(kda::SimtSmem<D>);
+    auto kern = kda::chunk_fwd_simt_kernel<T, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kern<<<(unsigned)(N * H), 256, smem, s>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)g,
+        (const T *)beta, h0, cu, N, (long)T_tot, H, (T *)o, hT);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <typename T>
+kda_status dispatch_simt(int d, const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *h0,
+                         const int32_t *cu, int N, int64_t T_tot, int H,
+                         void *o, float *hT, cudaStream_t s) {
+    switch (d) {
+    case 16: return launch_simt<T, 16>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
+    case 32: return launch_simt<T, 32>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
+    case 64: return launch_simt<T, 64>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
+    case 128: return launch_simt<T, 128>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
+    default: return KDA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int D, int SPLIT>
+kda_status launch_decode(const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, float *S, void *o,
+                         long units, cudaStream_t s) {
+    using Sh = kda::DecodeShape<D, SPLIT>;
+    const long blocks = (units + Sh::kHeadsPerBlock - 1) / Sh::kHeadsPerBlock;
+    kda::decode_step_kernel<T, D, SPLIT><<<(unsigned)blocks, Sh::kThreads, 0, s>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)g,
+        (const T *)beta, S, (T *)o, units);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <typename T>
+kda_status dispatch_decode(int d, const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S, void *o,
+                           long units, cudaStream_t s) {
+    switch (d) {
+    case 16: return launch_decode<T, 16, 1>(q, k, v, g, beta, S, o, units, s);
+    case 32: return launch_decode<T, 32, 1>(q, k, v, g, beta, S, o, units, s);
+    case 64: return launch_decode<T, 64, 1>(q, k, v, g, beta, S, o, units, s);
+    case 128: return launch_decode<T, 128, 2>(q, k, v, g, beta, S, o, units, s);
+    default: return KDA_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kda_version(void) { return 10000; }
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported dtype or head size";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+    case KDA_ERR_CUDA: return "CUDA runtime error";
+    case KDA_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+    case KDA_ERR_BAD_SEQLENS: return "malformed cu_seqlens";
+    }
+    return "unknown status";
+}
+
+size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t T_tot, int32_t H,
+                                    int32_t dk, int32_t dv, kda_dtype dt) {
+    if (N <= 0 || T_tot < 0 || H <= 0 || dk != dv) return 0;
+    if (dt == KDA_BF16 && dk == 128)
+        return kda::sm100_workspace_bytes(N, T_tot, H);
+    return 0;
+}
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *h0,
+                         const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                         void *o, float *hT, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    if (N < 0 || T_tot < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
+    if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
+    if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return T_tot == 0 ? KDA_OK : KDA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens == nullptr && (T_tot % N) != 0) return KDA_ERR_INVALID_ARGUMENT;
+    if ((int64_t)N * H > 0x7fffffff) return KDA_ERR_INVALID_ARGUMENT;
+    if (T_tot > 0) {
+        const void *req[] = {q, k, v, g, beta, o};
+        for (const void *p : req)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if ((h0 && !aligned16(h0)) || (hT && !aligned16(hT)) ||
+        (cu_seqlens && !aligned16(cu_seqlens)))
+        return KDA_ERR_INVALID_ARGUMENT;
+    const size_t ws_need = kda_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dt);
+    if (ws_need > 0 && (workspace == nullptr || workspace_bytes < ws_need ||
+                        (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return KDA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    if (dt == KDA_BF16)
+        return dispatch_simt<__nv_bfloat16>(dk, q, k, v, g, beta, h0, cu_seqlens,
+                                            N, T_tot, H, o, hT, s);
+    return dispatch_simt<float>(dk, q, k, v, g, beta, h0, cu_seqlens, N, T_tot,
+                                H, o, hT, s);
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S, void *o,
+                           int32_t B, int32_t H, int32_t dk, int32_t dv,
+                           kda_dtype dt, void *stream) {
+    if (B < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
+    if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
+    if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
+    if (B == 0) return KDA_OK;
+    const void *req[] = {q, k, v, g, beta, S, o};
+    for (const void *p : req)
+        if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const long units = (long)B * H;
+    if (dt == KDA_BF16)
+        return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, units, s);
+    return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, units, s);
+}
+
+kda_status kda_stream_status(void *stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, kda::g_status_word, sizeof(word)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(kda::g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
+    if (word & kda::kErrTimeout) return KDA_ERR_TIMEOUT;
+    if (word & kda::kErrSeqlens) return KDA_ERR_BAD_SEQLENS;
+    return KDA_OK;
+}
+
+}  // extern "C"

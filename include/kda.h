@@ -1,0 +1,147 @@
+/*
+ * kda.h -- C ABI of libkda, the Kimi Delta Attention (KDA) operator on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operator (per head, per sequence; pages on Kimi K3):
+ *
+ *   log a_t = -5 * sigmoid(g_t)                    per key channel
+ *   S_t     = Diag(a_t) S_{t-1}
+ *             + beta_t k_t (v_t - (Diag(a_t) S_{t-1})^T k_t)^T
+ *   o_t     = S_t^T q_t
+ *
+ *   "Kimi K3 发布核实与 Moonshot AI 主干架构演变" (dllmharness report), §3,
+ *   "KDA 为什么不同于 MLA": a per-head state matrix; the per-channel
+ *   retention alpha decays the old state first, the write strength beta with
+ *   the current key and value then corrects it, and the query reads the
+ *   updated state; training uses a form that is recurrent across chunks and
+ *   parallel within a chunk.  Same page, "K3 对 Kimi Linear 的进一步修改",
+ *   bullet 1: log-decay is a scaled sigmoid bounded below by -5, which keeps
+ *   the reciprocal scaling inside a 16-token tile within BF16 range.
+ *   "Kimi K3 模型架构解析：KDA、AttnRes 与 Stable LatentMoE", §二.2:
+ *   S_t = Update(S_{t-1}, k_t, v_t), o_t = Read(S_t, q_t); §二.3: 96 heads,
+ *   128-dimensional state channels per head.
+ *
+ * Conventions shared by every entry point
+ *   - All tensors are dense and row-major (last index contiguous) in the
+ *     layouts given below; every pointer must be 16-byte aligned.
+ *   - Pointers named "device" must point to device memory of the current
+ *     device.  The library never allocates: the caller owns every buffer,
+ *     including the workspace.
+ *   - q, k, v, g, beta and o share one element type (kda_dtype).  States
+ *     (h0, hT, S) are always fp32.
+ *   - g is the raw gate; the library applies log a = -5 sigmoid(g) itself.
+ *     beta is already the write strength in [0, 1].  No query scale is
+ *     applied (o = S^T q exactly).
+ *   - Argument errors are detected on the host before any launch: nothing is
+ *     written and nothing is launched.  Work is asynchronous on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream).  Errors found by a
+ *     kernel (malformed cu_seqlens, a bounded wait that ran out) set a
+ *     per-device status word that kda_stream_status() reports.
+ *   - Support: KDA_BF16 with dk = dv = 128 runs the tcgen05 tensor-core
+ *     path; KDA_BF16 with dk = dv in {16, 32, 64} and KDA_FP32 with
+ *     dk = dv in {16, 32, 64, 128} run an fp32 CUDA-core path (the fp32 test
+ *     mode).  Anything else returns KDA_ERR_UNSUPPORTED.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size     */
+    KDA_ERR_UNSUPPORTED = 2,      /* dtype / head size not in the matrix   */
+    KDA_ERR_WORKSPACE = 3,        /* workspace missing or too small        */
+    KDA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed  */
+    KDA_ERR_TIMEOUT = 5,          /* a kernel's bounded wait ran out       */
+    KDA_ERR_BAD_SEQLENS = 6       /* a kernel found cu_seqlens malformed   */
+} kda_status;
+
+typedef enum {
+    KDA_BF16 = 0,
+    KDA_FP32 = 1
+} kda_dtype;
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for these sizes (0 when it
+ * needs none).  Pure host function; never fails (returns 0 for sizes that
+ * kda_chunk_fwd would reject).
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t T_tot, int32_t H,
+                                    int32_t dk, int32_t dv, kda_dtype dt);
+
+/*
+ * Chunked prefill (16-token chunks: parallel inside a chunk, recurrent
+ * across chunks) over N packed sequences.
+ *
+ *   q, k, g     device [T_tot, H, dk]      (dt)
+ *   v           device [T_tot, H, dv]      (dt)
+ *   beta        device [T_tot, H]          (dt)
+ *   h0          device [N, H, dk, dv] fp32 initial states, or NULL (= 0)
+ *   cu_seqlens  device int32 [N+1], cu[0] = 0, non-decreasing, cu[N] = T_tot;
+ *               sequence n owns tokens [cu[n], cu[n+1]).  NULL means N
+ *               sequences of T_tot / N tokens each (T_tot % N must be 0).
+ *               Zero-length sequences are allowed (hT = h0).
+ *   o           device [T_tot, H, dv]      (dt) output, o_t = S_t^T q_t
+ *   hT          device [N, H, dk, dv] fp32 final states, or NULL (not
+ *               written).  hT may alias h0 exactly (in-place carry).
+ *   workspace   device scratch of kda_chunk_fwd_workspace_size() bytes
+ *               (may be NULL when that is 0); 256-byte aligned.
+ *
+ * Returns KDA_OK once the work is enqueued on `stream`.  Malformed
+ * cu_seqlens contents are found on the device: the affected sequences are
+ * skipped and kda_stream_status() returns KDA_ERR_BAD_SEQLENS.
+ */
+KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *h0,
+                         const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                         void *o, float *hT, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * One decode step for B sequences x H heads: one token each.  Same
+ * recurrence as the prefill (one token of it); S is updated in place.
+ *
+ *   q, k, g     device [B, H, dk]     (dt)
+ *   v           device [B, H, dv]     (dt)
+ *   beta        device [B, H]         (dt)
+ *   S           device [B, H, dk, dv] fp32, read and overwritten
+ *   o           device [B, H, dv]     (dt) output, read from the updated S
+ *
+ * A single pass over S: every state element is read once and written once.
+ */
+KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S,
+                           void *o, int32_t B, int32_t H, int32_t dk,
+                           int32_t dv, kda_dtype dt, void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's
+ * status word: KDA_OK, KDA_ERR_TIMEOUT, KDA_ERR_BAD_SEQLENS, or
+ * KDA_ERR_CUDA if the synchronisation itself failed.
+ */
+KDA_API kda_status kda_stream_status(void *stream);
+
+/* Static English description of a status code (never NULL). */
+KDA_API const char *kda_status_string(kda_status s);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+KDA_API int32_t kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

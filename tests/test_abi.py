@@ -1,0 +1,124 @@
+"""Host-only checks of the C ABI (no GPU needed).
+
+The library must load, export every entry point include/kda.h declares, and
+reject bad arguments on the host before touching the GPU: these calls pass
+null or misaligned pointers and must return the documented status without
+any CUDA call being made.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_60_b200 as kda
+from gated_delta_rule_60_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def _declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", text)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = _declared_symbols()
+    for must in ("kda_chunk_fwd", "kda_decode_step", "kda_stream_status",
+                 "kda_status_string", "kda_chunk_fwd_workspace_size",
+                 "kda_version"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert kda.kda_version() >= 10000
+    for s in range(7):
+        assert kda.kda_status_string(s)
+    assert kda.kda_status_string(99) == "unknown status"
+
+
+def test_workspace_size_is_host_only(lib):
+    assert lib.kda_chunk_fwd_workspace_size(0, 0, 1, 128, 128, 0) == 0
+    assert lib.kda_chunk_fwd_workspace_size(1, 64, 2, 16, 16, 1) == 0
+    ws = lib.kda_chunk_fwd_workspace_size(1, 8192, 96, 128, 128, 0)
+    assert ws >= 0
+
+
+def _call_fwd(lib, **over):
+    args = dict(q=16, k=16, v=16, g=16, beta=16, h0=None, cu=None, N=1, T=32,
+                H=2, dk=16, dv=16, dt=1, o=16, hT=None, ws=None, wsb=0,
+                stream=None)
+    args.update(over)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.kda_chunk_fwd(P(args["q"]), P(args["k"]), P(args["v"]),
+                             P(args["g"]), P(args["beta"]), P(args["h0"]),
+                             P(args["cu"]), args["N"], args["T"], args["H"],
+                             args["dk"], args["dv"], args["dt"], P(args["o"]),
+                             P(args["hT"]), P(args["ws"]), args["wsb"],
+                             P(args["stream"]))
+
+
+def test_chunk_fwd_host_validation(lib):
+    E = binding
+    assert _call_fwd(lib, q=None) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, o=None) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, k=24) == E.KDA_ERR_INVALID_ARGUMENT      # misaligned
+    assert _call_fwd(lib, h0=8) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, N=-1) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, H=0) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, T=-5) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, N=3, T=32) == E.KDA_ERR_INVALID_ARGUMENT  # 32 % 3
+    assert _call_fwd(lib, dk=48, dv=48) == E.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(lib, dk=16, dv=32) == E.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(lib, dt=7) == E.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(lib, N=0, T=0) == E.KDA_OK                    # nothing to do
+    assert _call_fwd(lib, N=0, T=4) == E.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_chunk_fwd_workspace_validation(lib):
+    need = lib.kda_chunk_fwd_workspace_size(1, 8192, 96, 128, 128, 0)
+    if need == 0:
+        pytest.skip("this configuration needs no workspace")
+    st = _call_fwd(lib, T=8192, H=96, dk=128, dv=128, dt=0, ws=None, wsb=0)
+    assert st == binding.KDA_ERR_WORKSPACE
+    st = _call_fwd(lib, T=8192, H=96, dk=128, dv=128, dt=0, ws=256, wsb=need - 1)
+    assert st == binding.KDA_ERR_WORKSPACE
+
+
+def test_decode_host_validation(lib):
+    P = ctypes.c_void_p
+    ok = [P(16)] * 7
+    def call(ptrs, B=2, H=2, dk=16, dv=16, dt=1):
+        return lib.kda_decode_step(*ptrs, B, H, dk, dv, dt, None)
+    bad = list(ok); bad[5] = None
+    assert call(bad) == binding.KDA_ERR_INVALID_ARGUMENT
+    bad = list(ok); bad[0] = P(20)
+    assert call(bad) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert call(ok, dk=100, dv=100) == binding.KDA_ERR_UNSUPPORTED
+    assert call(ok, B=-1) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert call(ok, B=0) == binding.KDA_OK
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = binding._lib
+    binding._lib = None
+    try:
+        with pytest.raises(ImportError):
+            binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        binding._lib = saved
