@@ -1,0 +1,413 @@
+"""Benchmark of the KDA hot path on B200.
+
+One step = one kda_chunk_fwd over the K3-shaped prefill workload
+(B=1, H=96, T=8192, d=128, bf16 inputs, fp32 state, S0=0): every row of the
+prefill path (tile loads, gate and decay scaling, intra-chunk transform,
+chunk products, state scan, output stores) runs inside the timed region.
+The decode workload (256 sequences x 96 heads, fp32 state, one
+kda_decode_step per step) is timed in the same run and reported under
+"decode".
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+For N > 1 launch under torch.distributed.run: every rank runs the same
+per-GPU workload on its own GPU (weak scaling; heads and sequences are
+independent, so there is no collective on the data path); the step time is
+the max over ranks.
+
+Timing: CUDA events on the stream the kernels are launched on, a barrier and
+a synchronize on both sides of the timed region, inputs (about 1 GB) larger
+than L2 so no flush is needed.  SM clocks are sampled with nvidia-smi during
+the timed region.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "KDA prefill Mtok/s (H=96,d=128,bf16) + % roofline; decode tok/s + HBM GB/s"
+
+# algorithmic bytes per (token, head) for bf16 q, k, v, g in, o out, beta
+BYTES_PER_TOKEN_HEAD = (4 * 128 + 128) * 2 + 2          # 1282
+FLOPS_PER_TOKEN_HEAD = 2 * 128 * 128 * 3 + 2 * 16 * 128 * 5   # 118,784
+STATE_BYTES = 128 * 128 * 4
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="kda_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap")
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist_init(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _oracle_sample(seconds_target=12.0):
+    """Time the fp64 oracle on a bounded sample of the K3 workload: a few
+    heads over the full 8192 tokens.  Returns (tokens/s full-H equivalent,
+    cores, sample description)."""
+    import oracle
+    from gated_delta_rule_60_b200 import workloads
+    w = workloads.K3_PREFILL
+    cores = oracle.threads()
+    heads = max(1, min(w.H, cores))
+    inp = w.make()
+    q, k, v, g, b = (x[:, :heads].contiguous() for x in (inp.q, inp.k, inp.v,
+                                                          inp.g, inp.beta))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.forward(q, k, v, g, b, inp.cu_seqlens, None)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds_target or reps >= 64:
+            break
+    dt = time.perf_counter() - t0
+    token_heads = reps * heads * w.T_tot
+    tok_s = token_heads / w.H / dt
+    return tok_s, cores, ("%d of 96 heads x 8192 tokens, %d pass(es), %.1f s; "
+                          "value in full-96-head tokens/s" % (heads, reps, dt))
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from gated_delta_rule_60_b200 import workloads
+    w = workloads.K3_PREFILL
+    cores = oracle.threads()
+    heads = max(1, min(w.H, cores))
+    inp = w.make()
+    q, k, v, g, b = (x[:, :heads].contiguous() for x in (inp.q, inp.k, inp.v,
+                                                          inp.g, inp.beta))
+    for _ in range(args.warmup):
+        oracle.forward(q[:256], k[:256], v[:256], g[:256], b[:256], [0, 256], None)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(q, k, v, g, b, inp.cu_seqlens, None)
+        times.append(time.perf_counter() - t0)
+    dt = statistics.median(times)
+    value = heads * w.T_tot / w.H / dt / 1e6
+    sample = "%d of 96 heads x 8192 tokens per step (full-96-head tokens/s)" % heads
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "k3_prefill B=1 H=96 T=8192 d=128 bf16 S0=0 "
+                               "(oracle on a head sample)"},
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_gpu(args):
+    from gated_delta_rule_60_b200 import binding, inputs, workloads
+
+    world, rank, local = _dist_init(args.gpus)
+    dev = torch.device("cuda", local)
+    binding.load_library()
+    hbm_peak, tc_peak, peak_kind = _peaks()
+
+    # ---------------- prefill workload ----------------
+    w = workloads.K3_PREFILL
+    inp = w.make()
+    T, H, d = w.T_tot, w.H, w.dk
+    dq, dk_, dv_, dg, db = (x.to(dev) for x in (inp.q, inp.k, inp.v, inp.g, inp.beta))
+    cu = inp.cu_seqlens.to(dev)
+    o = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+    hT = torch.empty(1, H, d, d, dtype=torch.float32, device=dev)
+    ws_n = binding.kda_chunk_fwd_workspace_size(1, T, H, d, d, torch.bfloat16)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev) if ws_n else None
+    stream = torch.cuda.Stream(device=dev)
+    launches_per_step = 1
+
+    def step():
+        binding.kda_chunk_fwd(dq, dk_, dv_, dg, db, None, cu, o=o, hT=hT,
+                              workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            step()
+    stream.synchronize()
+    assert binding.kda_stream_status(stream) == binding.KDA_OK
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    _barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev[0].record(stream)
+            for i in range(args.steps):
+                step()
+                ev[i + 1].record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    _barrier(world)
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms = _max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    st = binding.kda_stream_status(stream)
+    if st != binding.KDA_OK:
+        raise RuntimeError("kernel status: " + binding.kda_status_string(st))
+    clocks = clk.summary()
+
+    alg_bytes = T * H * BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    kern_ms = statistics.mean(per_launch)
+    achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+    value = world * T / (ms_step * 1e-3) / 1e6
+
+    # ---------------- end to end, host buffers ----------------
+    host = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    o_host = torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory()
+    h_host = torch.empty(1, H, d, d, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_host.numel() * 2 + h_host.numel() * 4
+
+    def e2e_step():
+        xs = {n: t.to(dev, non_blocking=True) for n, t in host.items()}
+        binding.kda_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"],
+                              None, cu, o=o, hT=hT, workspace=ws, stream=stream)
+        o_host.copy_(o, non_blocking=True)
+        h_host.copy_(hT, non_blocking=True)
+
+    e2e_steps = max(2, min(args.steps, 10))
+    with torch.cuda.stream(stream):
+        e2e_step()
+        stream.synchronize()
+        _barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+    stream.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_val = world * T / (e2e_ms * 1e-3) / 1e6
+    del host
+
+    # ---------------- decode workload ----------------
+    B, Hd, D = workloads.DECODE_B, workloads.DECODE_H, workloads.DECODE_D
+    # the state: a 512-token prefill of every sequence (drawn on the device)
+    pre = inputs.make_prefill([workloads.DECODE_PREFILL] * B, Hd, D, D,
+                              torch.bfloat16, workloads.DECODE_SEED, device=dev)
+    S = torch.empty(B, Hd, D, D, dtype=torch.float32, device=dev)
+    od_pre = torch.empty(B * workloads.DECODE_PREFILL, Hd, D, dtype=torch.bfloat16,
+                         device=dev)
+    ws_pre_n = binding.kda_chunk_fwd_workspace_size(
+        B, B * workloads.DECODE_PREFILL, Hd, D, D, torch.bfloat16)
+    ws_pre = torch.empty(ws_pre_n, dtype=torch.uint8, device=dev) if ws_pre_n else None
+    binding.kda_chunk_fwd(pre.q, pre.k, pre.v, pre.g, pre.beta, None,
+                          pre.cu_seqlens, o=od_pre, hT=S, workspace=ws_pre,
+                          stream=stream)
+    stream.synchronize()
+    del pre, od_pre, ws_pre
+    xs = [inputs.make_decode_step(B, Hd, D, D, torch.bfloat16,
+                                  workloads.DECODE_STEP_SEED0 + s, device=dev)
+          for s in range(4)]
+    xs = [{n: getattr(x, n) for n in ("q", "k", "v", "g", "beta")} for x in xs]
+    od = torch.empty(B, Hd, D, dtype=torch.bfloat16, device=dev)
+
+    def dstep(i):
+        x = xs[i % len(xs)]
+        binding.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S,
+                                o=od, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            dstep(i)
+    stream.synchronize()
+    dsteps = max(args.steps, 10)
+    dev_ev = [torch.cuda.Event(enable_timing=True) for _ in range(dsteps + 1)]
+    _barrier(world)
+    with torch.cuda.stream(stream):
+        dev_ev[0].record(stream)
+        for i in range(dsteps):
+            dstep(i)
+            dev_ev[i + 1].record(stream)
+    stream.synchronize()
+    dms = [dev_ev[i].elapsed_time(dev_ev[i + 1]) for i in range(dsteps)]
+    d_ms = _max_over_ranks(statistics.median(dms), world)
+    d_bytes = 2 * B * Hd * D * D * 4 + B * Hd * (4 * D + D) * 2 + B * Hd * 2
+    d_gbs = d_bytes / (d_ms * 1e-3) / 1e9
+    assert binding.kda_stream_status(stream) == binding.KDA_OK
+
+    if rank != 0:
+        _barrier(world)
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tok_s, cores, sample = _oracle_sample()
+        cpu = {"value": tok_s / 1e6, "unit": "Mtok/s", "cores": cores,
+               "kind": "oracle", "sample": sample}
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "Mtok/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "k3_prefill B=1 H=96 T=8192 d=128 bf16 S0=0, "
+                               "chunk 16, one kda_chunk_fwd per step",
+                   "tokens_per_gpu": T, "heads": H, "head_dim": d,
+                   "l2": "inputs ~1 GB > L2 (126 MB), no flush",
+                   "parallelism": "replicas: independent heads/sequences per GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "kernel_ms": kern_ms,
+                     "tensor_tflops": T * H * FLOPS_PER_TOKEN_HEAD / (kern_ms * 1e-3) / 1e12,
+                     "tensor_peak_tflops": tc_peak},
+        "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "decode": {"workload": "256 seqs x 96 heads, d=128, fp32 state, one "
+                               "kda_decode_step per step",
+                   "tok_s": B / (d_ms * 1e-3), "ms_per_step": d_ms,
+                   "hbm_gbs": d_gbs, "frac_of_peak": d_gbs / hbm_peak,
+                   "algorithmic_bytes_per_step": d_bytes},
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "gpu_launches": args.steps * launches_per_step,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+    if world > 1:
+        _barrier(world)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="libkda", choices=["libkda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    rc = run_gpu(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

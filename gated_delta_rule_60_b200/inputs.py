@@ -48,22 +48,31 @@ def cu_from_lengths(lengths) -> torch.Tensor:
 
 
 def make_prefill(lengths, H: int, dk: int, dv: int, dtype=torch.bfloat16,
-                 seed: int = 0, h0_std: Optional[float] = None
-                 ) -> PrefillInputs:
-    """Packed varlen prefill inputs for sequences of the given lengths."""
-    gen = torch.Generator().manual_seed(int(seed))
+                 seed: int = 0, h0_std: Optional[float] = None,
+                 device=None) -> PrefillInputs:
+    """Packed varlen prefill inputs for sequences of the given lengths.
+
+    With ``device`` set, the numbers are drawn by that device's generator
+    (same distributions, a different random stream) and stay there; this is
+    for large benchmark inputs that would be slow to draw on the CPU."""
+    dev = torch.device("cpu") if device is None else torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(int(seed))
     T = int(sum(lengths))
     N = len(lengths)
-    q = _unit_rows(torch.randn(T, H, dk, generator=gen))
-    k = _unit_rows(torch.randn(T, H, dk, generator=gen))
-    v = torch.randn(T, H, dv, generator=gen)
-    g = torch.randn(T, H, dk, generator=gen)
-    beta = torch.sigmoid(torch.randn(T, H, generator=gen))
+    kw = dict(generator=gen, device=dev)
+
+    def draw_unit(*shape):
+        return _unit_rows(torch.randn(*shape, **kw)).to(dtype)
+
+    q = draw_unit(T, H, dk)
+    k = draw_unit(T, H, dk)
+    v = torch.randn(T, H, dv, **kw).to(dtype)
+    g = torch.randn(T, H, dk, **kw).to(dtype)
+    beta = torch.sigmoid(torch.randn(T, H, **kw)).to(dtype)
     h0 = None
     if h0_std is not None:
-        h0 = torch.randn(N, H, dk, dv, generator=gen) * float(h0_std)
-    return PrefillInputs(q.to(dtype), k.to(dtype), v.to(dtype), g.to(dtype),
-                         beta.to(dtype), h0, cu_from_lengths(lengths))
+        h0 = torch.randn(N, H, dk, dv, **kw) * float(h0_std)
+    return PrefillInputs(q, k, v, g, beta, h0, cu_from_lengths(lengths).to(dev))
 
 
 def draw_lengths(n: int, lo: int, hi: int, seed: int) -> List[int]:
@@ -82,14 +91,16 @@ class DecodeInputs:
 
 
 def make_decode_step(B: int, H: int, dk: int, dv: int, dtype=torch.bfloat16,
-                     seed: int = 0) -> DecodeInputs:
+                     seed: int = 0, device=None) -> DecodeInputs:
     """One token per (sequence, head) with the prefill distributions."""
-    gen = torch.Generator().manual_seed(int(seed))
-    q = _unit_rows(torch.randn(B, H, dk, generator=gen))
-    k = _unit_rows(torch.randn(B, H, dk, generator=gen))
-    v = torch.randn(B, H, dv, generator=gen)
-    g = torch.randn(B, H, dk, generator=gen)
-    beta = torch.sigmoid(torch.randn(B, H, generator=gen))
+    dev = torch.device("cpu") if device is None else torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(int(seed))
+    kw = dict(generator=gen, device=dev)
+    q = _unit_rows(torch.randn(B, H, dk, **kw))
+    k = _unit_rows(torch.randn(B, H, dk, **kw))
+    v = torch.randn(B, H, dv, **kw)
+    g = torch.randn(B, H, dk, **kw)
+    beta = torch.sigmoid(torch.randn(B, H, **kw))
     return DecodeInputs(q.to(dtype), k.to(dtype), v.to(dtype), g.to(dtype),
                         beta.to(dtype))
 
