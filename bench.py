@@ -227,6 +227,7 @@ def run_gpu(args):
     ws_n = binding.kda_chunk_fwd_workspace_size(1, T, H, d, d, torch.bfloat16)
     ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev) if ws_n else None
     stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
     launches_per_step = 1
 
     def step():
@@ -266,6 +267,17 @@ def run_gpu(args):
     value = world * T / (ms_step * 1e-3) / 1e6
 
     # ---------------- end to end, host buffers ----------------
+    e2e = None
+    if not args.skip_e2e:
+        e2e = _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding)
+    decode = None
+    if not args.skip_decode:
+        decode = _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads)
+    return _report(args, world, rank, value, ms_step, achieved, hbm_peak, peak_kind, alg_bytes,
+                   kern_ms, T, H, d, tc_peak, e2e, decode, clocks, launches_per_step)
+
+
+def _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding):
     host = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
     o_host = torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory()
     h_host = torch.empty(1, H, d, d, dtype=torch.float32).pin_memory()
@@ -292,13 +304,16 @@ def run_gpu(args):
     stream.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e_val = world * T / (e2e_ms * 1e-3) / 1e6
-    del host
+    return {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
 
-    # ---------------- decode workload ----------------
+
+def _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads):
     B, Hd, D = workloads.DECODE_B, workloads.DECODE_H, workloads.DECODE_D
     # the state: a 512-token prefill of every sequence (drawn on the device)
     pre = inputs.make_prefill([workloads.DECODE_PREFILL] * B, Hd, D, D,
                               torch.bfloat16, workloads.DECODE_SEED, device=dev)
+    torch.cuda.synchronize()
     S = torch.empty(B, Hd, D, D, dtype=torch.float32, device=dev)
     od_pre = torch.empty(B * workloads.DECODE_PREFILL, Hd, D, dtype=torch.bfloat16,
                          device=dev)
@@ -314,6 +329,7 @@ def run_gpu(args):
                                   workloads.DECODE_STEP_SEED0 + s, device=dev)
           for s in range(4)]
     xs = [{n: getattr(x, n) for n in ("q", "k", "v", "g", "beta")} for x in xs]
+    torch.cuda.synchronize()
     od = torch.empty(B, Hd, D, dtype=torch.bfloat16, device=dev)
 
     def dstep(i):
@@ -339,7 +355,15 @@ def run_gpu(args):
     d_bytes = 2 * B * Hd * D * D * 4 + B * Hd * (4 * D + D) * 2 + B * Hd * 2
     d_gbs = d_bytes / (d_ms * 1e-3) / 1e9
     assert binding.kda_stream_status(stream) == binding.KDA_OK
+    return {"workload": "256 seqs x 96 heads, d=128, fp32 state built by a 512-token "
+                        "prefill, one kda_decode_step per step",
+            "tok_s": world * B / (d_ms * 1e-3), "ms_per_step": d_ms,
+            "hbm_gbs": d_gbs, "frac_of_peak": d_gbs / hbm_peak,
+            "algorithmic_bytes_per_step": d_bytes}
 
+
+def _report(args, world, rank, value, ms_step, achieved, hbm_peak, peak_kind, alg_bytes,
+            kern_ms, T, H, d, tc_peak, e2e, decode, clocks, launches_per_step):
     if rank != 0:
         _barrier(world)
         return 0
@@ -375,13 +399,8 @@ def run_gpu(args):
                      "kernel_ms": kern_ms,
                      "tensor_tflops": T * H * FLOPS_PER_TOKEN_HEAD / (kern_ms * 1e-3) / 1e12,
                      "tensor_peak_tflops": tc_peak},
-        "e2e": {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "decode": {"workload": "256 seqs x 96 heads, d=128, fp32 state, one "
-                               "kda_decode_step per step",
-                   "tok_s": B / (d_ms * 1e-3), "ms_per_step": d_ms,
-                   "hbm_gbs": d_gbs, "frac_of_peak": d_gbs / hbm_peak,
-                   "algorithmic_bytes_per_step": d_bytes},
+        "e2e": e2e,
+        "decode": decode,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "gpu_launches": args.steps * launches_per_step,
         "cpu_baseline": cpu,
@@ -399,6 +418,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="libkda", choices=["libkda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--skip-decode", action="store_true",
+                    help="skip the decode measurement")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

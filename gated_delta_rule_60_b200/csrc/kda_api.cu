@@ -130,6 +130,11 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
         return KDA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
+    if (dt == KDA_BF16 && dk == 128)
+        return T_tot == 0 && hT == nullptr
+                   ? KDA_OK
+                   : kda::sm100_chunk_fwd(q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H,
+                                          o, hT, workspace, s);
     if (dt == KDA_BF16)
         return dispatch_simt<__nv_bfloat16>(dk, q, k, v, g, beta, h0, cu_seqlens,
                                             N, T_tot, H, o, hT, s);
@@ -154,6 +159,20 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
         return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, units, s);
     return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, units, s);
 }
+
+#ifdef KDA_TRACE
+// Profiling builds only: copy the stage timestamps of the traced chain out.
+KDA_API int kda_debug_trace_read(unsigned long long *dst, size_t n) {
+    const size_t bytes = sizeof(kda::prefill::g_trace);
+    if (n * sizeof(unsigned long long) < bytes) return -1;
+    return cudaMemcpyFromSymbol(dst, kda::prefill::g_trace, bytes) == cudaSuccess ? 0 : -1;
+}
+KDA_API int kda_debug_cta_times(unsigned long long *dst, size_t n) {
+    const size_t bytes = sizeof(kda::prefill::g_cta_time);
+    if (n * sizeof(unsigned long long) < bytes) return -1;
+    return cudaMemcpyFromSymbol(dst, kda::prefill::g_cta_time, bytes) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 kda_status kda_stream_status(void *stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -25,6 +25,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace kda {
@@ -69,14 +70,66 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` polls (each poll may suspend the
-// thread briefly) or as soon as *abort is set.  Returns true on success.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity,
+                                                   uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// How a bounded wait polls: 0 = try_wait (the hardware may suspend the
+// thread between polls), 1 = test_wait spin, 2 = try_wait with a short
+// suspend-time hint, 3 = test_wait with a short sleep between polls.
+#ifndef KDA_MBAR_WAIT
+#define KDA_MBAR_WAIT 0
+#endif
+
+__device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity) {
+#if KDA_MBAR_WAIT == 1
+    return mbar_test_wait(bar, parity);
+#elif KDA_MBAR_WAIT == 3
+    if (mbar_test_wait(bar, parity)) return true;
+    __nanosleep(32);
+    return false;
+#elif KDA_MBAR_WAIT == 2
+    return mbar_try_wait_hint(bar, parity, 64);
+#else
+    return mbar_try_wait(bar, parity);
+#endif
+}
+
+// Bounded wait: gives up once `limit_cycles` SM clock cycles have passed
+// since the first unsuccessful poll, or as soon as *abort is set.  Returns
+// true on success.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort, uint32_t limit) {
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u && *abort) return false;
-        if (it >= limit) return false;
+                                          volatile int *abort,
+                                          unsigned long long limit_cycles) {
+    if (mbar_poll(bar, parity)) return true;
+    const unsigned long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_poll(bar, parity)) return true;
+        if ((it & 63u) == 0u) {
+            if (*abort) return false;
+            if (clock64() - t0 > limit_cycles) return false;
+        }
     }
 }
 
@@ -156,6 +209,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, tf32 inputs (32-bit A columns)
+__device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -228,6 +292,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// tf32 x tf32 -> f32 (kind::tf32), same field layout as idesc_bf16.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of fp32 element (row, col) of a [rows][32] fp32 region in the
+// 128B-swizzled layout (32 elements per 128-byte row).
+__host__ __device__ __forceinline__ uint32_t sw128_off32(uint32_t row, uint32_t col) {
+    return (row >> 3) * 1024u + (row & 7u) * 128u +
+           ((((col >> 2) ^ (row & 7u)) & 7u) << 4) + (col & 3u) * 4u;
+}
+
+// Byte offset of fp32 element (row, k) of a [16][16] fp32 K-major tile in the
+// no-swizzle core-matrix layout (8 rows x 16 B cores) with LBO = 128 (next
+// 4 k) and SBO = 512 (next 8 rows).
+__host__ __device__ __forceinline__ uint32_t core16_off32(uint32_t row, uint32_t k) {
+    return (row >> 3) * 512u + (k >> 2) * 128u + (row & 7u) * 16u + (k & 3u) * 4u;
+}
+
 // Byte offset of element (row, col) of a [rows][64] bf16 region in the
 // 128B-swizzled layout (the TMA SWIZZLE_128B box layout and the canonical
 // K-major / MN-major 128B-swizzle atom).  The region must be 1024-aligned.
@@ -241,6 +325,31 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t co
 // (next 8 rows).
 __host__ __device__ __forceinline__ uint32_t core16_off(uint32_t row, uint32_t k) {
     return (row >> 3) * 256u + (k >> 3) * 128u + (row & 7u) * 16u + (k & 7u) * 2u;
+}
+
+// Packed fp32 pair arithmetic (sm_100 f32x2 instructions).
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

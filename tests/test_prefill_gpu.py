@@ -194,3 +194,25 @@ def test_bad_seqlens_reported_not_faulted():
     binding.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, bad, o=o)
     assert binding.kda_stream_status() == binding.KDA_ERR_BAD_SEQLENS
     assert binding.kda_stream_status() == binding.KDA_OK  # cleared
+
+
+def test_long_sequence_segmented():
+    """One long sequence per head with few heads takes the segment-parallel
+    path (local pass, combine, final pass).  A ragged last segment and a
+    carried state; every unit checked against the oracle."""
+    T, H = 16384 + 77, 2
+    assert binding.kda_chunk_fwd_workspace_size(1, T, H, 128, 128, torch.bfloat16) > 0
+    inp = inputs.make_prefill([T], H, 128, 128, torch.bfloat16, seed=96, h0_std=0.02)
+    o, hT = run(inp)
+    check(inp, o, hT)
+
+
+def test_long_1m_workload_sampled():
+    """The long-context workload (T = 1,048,576, H = 16, bf16, S0 = 0): the
+    oracle runs 2 seeded heads over the full length."""
+    w = workloads.LONG
+    inp = w.make()
+    o, hT = run(inp)
+    mask = np.zeros((1, w.H), dtype=bool)
+    mask[0, np.random.default_rng(3).choice(w.H, 2, replace=False)] = True
+    check(inp, o, hT, unit_mask=mask)
