@@ -57,6 +57,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                   i32, ctypes.c_int, vp, vp, vp, sz, vp]
+    lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                          i32, ctypes.c_int, vp, vp, vp]
     lib.kda_decode_step.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
                                     i32, ctypes.c_int, vp]
@@ -159,6 +162,44 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                            ws_bytes, _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd")
+    return o, hT
+
+
+def kda_chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          g: torch.Tensor, beta: torch.Tensor,
+                          h0: Optional[torch.Tensor] = None,
+                          cu_seqlens: Optional[torch.Tensor] = None, *,
+                          o: torch.Tensor, hT: Optional[torch.Tensor] = None,
+                          num_seqs: Optional[int] = None,
+                          stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_chunk_fwd for callers that cannot allocate device memory: o (and
+    hT, if wanted) must be given; the long-sequence scratch comes from the
+    library's static device array, so nothing here allocates."""
+    lib = load_library()
+    dev = q.device
+    T_tot, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name, shp in ((q, "q", (T_tot, H, dk)), (k, "k", (T_tot, H, dk)),
+                         (g, "g", (T_tot, H, dk)), (v, "v", (T_tot, H, dv)),
+                         (beta, "beta", (T_tot, H)), (o, "o", (T_tot, H, dv))):
+        _check(t, name, dt, shp, dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                   _ptr(h0), _ptr(cu_seqlens), N, T_tot, H, dk, dv,
+                                   _DTYPES[dt], _ptr(o), _ptr(hT), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_noalloc")
     return o, hT
 
 

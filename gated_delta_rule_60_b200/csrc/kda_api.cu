@@ -191,3 +191,5 @@ kda_status kda_stream_status(void *stream) {
 }
 
 }  // extern "C"
+
+#include "kda_noalloc.cuh"

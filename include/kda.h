@@ -128,6 +128,33 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            int32_t dv, kda_dtype dt, void *stream);
 
 /*
+ * kda_chunk_fwd without a caller-provided workspace, for callers that cannot
+ * allocate device memory: a serving engine that has reserved nearly all of
+ * the GPU's memory for its own caches, a plugin whose host owns the
+ * allocator, or latency-sensitive code that must not call cudaMalloc because
+ * it can synchronise the device.  The pages have no counterpart; this is a
+ * convenience of the library.
+ *
+ * Arguments and results are those of kda_chunk_fwd (without workspace and
+ * workspace_bytes).  The scratch the long-sequence path needs (see
+ * kda_chunk_fwd_workspace_size) comes from a static device array of 16 MiB
+ * that every GPU loading libkda holds until the process exits; the call
+ * allocates nothing.  A problem that needs more scratch than that returns
+ * KDA_ERR_WORKSPACE before anything is launched.  The first call on a device
+ * looks up the array's device address; make that first call before any
+ * stream capture.  All calls on a device share the array: calls that may
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * it and must not be issued.  Every scratch value a call reads is written
+ * earlier in the same call, so leftover contents from an earlier call do not
+ * matter.
+ */
+KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                         const void *g, const void *beta, const float *h0,
+                                         const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                         void *o, float *hT, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's
  * status word: KDA_OK, KDA_ERR_TIMEOUT, KDA_ERR_BAD_SEQLENS, or
  * KDA_ERR_CUDA if the synchronisation itself failed.
