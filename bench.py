@@ -44,6 +44,27 @@ FLOPS_PER_TOKEN_HEAD = 2 * 128 * 128 * 3 + 2 * 16 * 128 * 5   # 118,784
 STATE_BYTES = 128 * 128 * 4
 
 
+def _measured_traffic():
+    """DRAM bytes per launch of the prefill kernel from the committed ncu
+    summary, or None when the kernel sources changed since that capture."""
+    import hashlib
+    srcs = [os.path.join(ROOT, "gated_delta_rule_60_b200", "csrc", f)
+            for f in ("kda_chunk_sm100.cuh", "sm100_ptx.cuh")]
+    try:
+        h = hashlib.sha256(b"".join(open(f, "rb").read() for f in srcs)).hexdigest()[:16]
+        text = open(os.path.join(ROOT, "profiles", "chunk_fwd_sm100_k3_prefill.md")).read()
+    except OSError:
+        return None
+    fields = dict(line.split(":", 1) for line in text.splitlines()
+                  if line.startswith(("kernel-source-sha256-16:", "traffic_bytes_per_launch:")))
+    if fields.get("kernel-source-sha256-16", "").strip() != h:
+        return None
+    val = fields.get("traffic_bytes_per_launch", "").strip().split()
+    if len(val) != 2 or val[1] != "kB":
+        return None
+    return float(val[0]) * 1e3
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -216,6 +237,14 @@ def run_gpu(args):
     binding.load_library()
     hbm_peak, tc_peak, peak_kind = _peaks()
 
+    if args.only == "decode":
+        stream = torch.cuda.Stream(device=dev)
+        torch.cuda.synchronize()
+        decode = _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads)
+        if rank == 0:
+            print(json.dumps({"only": "decode", "decode": decode}))
+        return 0
+
     # ---------------- prefill workload ----------------
     w = workloads.K3_PREFILL
     inp = w.make()
@@ -266,15 +295,65 @@ def run_gpu(args):
     achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
     value = world * T / (ms_step * 1e-3) / 1e6
 
+    if args.only == "prefill":
+        if rank == 0:
+            print(json.dumps({"only": "prefill", "ms": kern_ms, "Mtok_s": value,
+                              "hbm_frac": achieved / hbm_peak}))
+        return 0
+
     # ---------------- end to end, host buffers ----------------
     e2e = None
     if not args.skip_e2e:
         e2e = _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding)
+    del dq, dk_, dv_, dg, db, o
+    torch.cuda.empty_cache()
+    extra = {}
+    if not args.skip_workloads:
+        for wl in (workloads.VARLEN, workloads.LONG):
+            extra[wl.name] = _measure_workload(wl, dev, stream, args, world, hbm_peak, binding,
+                                               inputs)
+            torch.cuda.empty_cache()
     decode = None
     if not args.skip_decode:
         decode = _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads)
     return _report(args, world, rank, value, ms_step, achieved, hbm_peak, peak_kind, alg_bytes,
-                   kern_ms, T, H, d, tc_peak, e2e, decode, clocks, launches_per_step)
+                   kern_ms, T, H, d, tc_peak, e2e, decode, clocks, launches_per_step, extra)
+
+
+def _measure_workload(w, dev, stream, args, world, hbm_peak, binding, inputs):
+    """One prefill workload (drawn on the device), timed like the headline."""
+    pre = inputs.make_prefill(list(w.lengths), w.H, w.dk, w.dv, w.dtype, w.seed,
+                              w.h0_std, device=dev)
+    torch.cuda.synchronize()
+    N, T = len(w.lengths), w.T_tot
+    o = torch.empty(T, w.H, w.dv, dtype=w.dtype, device=dev)
+    hT = torch.empty(N, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+    ws_n = binding.kda_chunk_fwd_workspace_size(N, T, w.H, w.dk, w.dv, w.dtype)
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
+
+    def step():
+        binding.kda_chunk_fwd(pre.q, pre.k, pre.v, pre.g, pre.beta, pre.h0, pre.cu_seqlens,
+                              o=o, hT=hT, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    steps = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    assert binding.kda_stream_status(stream) == binding.KDA_OK
+    ms = _max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    alg = T * w.H * BYTES_PER_TOKEN_HEAD + N * w.H * STATE_BYTES * (2 if w.h0_std else 1)
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {"tokens": T, "heads": w.H, "sequences": N, "ms": ms,
+            "Mtok_s": world * T / (ms * 1e-3) / 1e6, "hbm_gbs": gbs,
+            "frac_of_peak": gbs / hbm_peak, "launches_per_step": 1 if not ws_n else 3}
 
 
 def _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding):
@@ -325,6 +404,7 @@ def _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloa
                           stream=stream)
     stream.synchronize()
     del pre, od_pre, ws_pre
+    torch.cuda.empty_cache()
     xs = [inputs.make_decode_step(B, Hd, D, D, torch.bfloat16,
                                   workloads.DECODE_STEP_SEED0 + s, device=dev)
           for s in range(4)]
@@ -363,7 +443,7 @@ def _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloa
 
 
 def _report(args, world, rank, value, ms_step, achieved, hbm_peak, peak_kind, alg_bytes,
-            kern_ms, T, H, d, tc_peak, e2e, decode, clocks, launches_per_step):
+            kern_ms, T, H, d, tc_peak, e2e, decode, clocks, launches_per_step, extra):
     if rank != 0:
         _barrier(world)
         return 0
@@ -394,13 +474,14 @@ def _report(args, world, rank, value, ms_step, achieved, hbm_peak, peak_kind, al
                    "parallelism": "replicas: independent heads/sequences per GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak,
                      "unit": "GB/s", "frac": achieved / hbm_peak,
-                     "traffic": None, "peak_source": peak_kind,
+                     "traffic": _measured_traffic(), "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "kernel_ms": kern_ms,
                      "tensor_tflops": T * H * FLOPS_PER_TOKEN_HEAD / (kern_ms * 1e-3) / 1e12,
                      "tensor_peak_tflops": tc_peak},
         "e2e": e2e,
         "decode": decode,
+        "workloads": extra,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "gpu_launches": args.steps * launches_per_step,
         "cpu_baseline": cpu,
@@ -422,6 +503,10 @@ def main():
                     help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--skip-decode", action="store_true",
                     help="skip the decode measurement")
+    ap.add_argument("--skip-workloads", action="store_true",
+                    help="skip the varlen and long-context prefill measurements")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part only (for profiling): the K3 prefill or the decode")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
