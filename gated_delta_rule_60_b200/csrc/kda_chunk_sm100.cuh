@@ -1,46 +1,50 @@
 // kda_chunk_sm100.cuh -- fused chunked KDA prefill on B200 tensor cores
-// (bf16 inputs, fp32 state, d_k = d_v = 128, 16-token chunks).
+// (bf16 inputs, fp32 state, d_k = d_v = 128).
 //
 // Operator (page "Kimi K3 发布核实与 Moonshot AI 主干架构演变", §3): per head
 // the state S (d_k x d_v) is decayed per key channel by a_t, corrected with
 // beta_t, k_t, v_t (delta rule) and read by q_t after the update; prefill uses
 // a form that is recurrent across chunks and parallel inside a chunk.  Same
 // page, "K3 对 Kimi Linear 的进一步修改" bullet 1: log a = -5 sigmoid(g), so the
-// cumulative log-decay inside a 16-token tile stays in [-80, 0] and the
-// reciprocal decay scaling fits BF16 range, letting every causal tile take
-// the dense-matrix path.
+// cumulative log-decay over a 16-token tile stays in [-80, 0] and reciprocal
+// decay scaling fits the BF16 exponent range.
 //
-// Chunk algorithm (16 rows r, start state S0, per key channel c):
-//   e_r = exp(b_r) = prod_{i<=r} a_i,  m = b_7 (centre), eps = e^m,
-//   delta = e^{b_15 - m}  (so the chunk decay is gamma = eps * delta)
-//   Kr = K e^{b-m},  Qr = Q e^{b-m},  Kh = K e^{m-b}      (|exponent| <= 40)
-//   A_kk = Kr Kh^T,  A_qk = Qr Kh^T
-//   T = (I + Diag(beta) strict_lower(A_kk))^-1 Diag(beta)
-//   W = T Kr Diag(eps),  U = T V - W S0
-//   O = (Q e^b) S0 + causal(A_qk) U
-//   S = Diag(delta) (Diag(eps) S0 + Kh^T U)
-// On the tensor cores everything is written transposed so that the 128
-// value channels are the MMA M dimension (TMEM lanes):
-//   W^T = Diag(eps) Kr^T T^T      U_v^T = V^T T^T           (M=128, N=16, K=16)
-//   [U | O]^T += S^T [-W ; Q e^b]^T                          (M=128, N=32, K=128)
-//   O^T += U^T causal(A_qk)^T,     Y = Diag(eps)S^T... + U^T Kh   (K=16)
-// The fp32 state stays in tensor memory as Y = (eps * S)^T plus the
-// accumulated U^T Kh; once per chunk the scan warpgroup turns it into
-// S = delta * Y, writes the bf16 copy the next chunk's MMA reads, and
-// stores the next chunk's eps * S back.  The two 16x16 intra products of a
-// chunk come from one M=128 MMA (K rows and Q rows of a 32-token batch
-// stacked on M).
+// Step algorithm.  The state advances in steps of two 16-token tiles (32
+// rows r, start state S0).  Per key channel, b_r is the cumulative log-decay
+// from the start of the step and the reference point is m = b_15, the end of
+// the first tile, so every scaled exponent lies within one tile's range
+// (|b_r - m| <= 80):
+//   eps = e^m,  delta = e^{b_31 - m},  gamma = eps * delta (step decay)
+//   Kr = K e^{b-m},  Qr = Q e^{b-m},  Kh = K e^{m-b}
+//   A_kk = Kr Kh^T,  A_qk = Qr Kh^T   (causal entries are e^{b_r - b_i} <= 1)
+//   T = (I + Diag(beta) strict_lower(A_kk))^-1 Diag(beta)     (32 x 32)
+//   P = causal(A_qk) T,   Z = Diag(delta) Kh^T T              (d_k x 32)
+// (T by forward substitution on the CUDA cores; every product on the tensor
+// cores.)
+// With Ke = Kr Diag(eps) = K e^b and Qe = Q e^b the step is exactly
+//   W = V - Ke S0,   S_next = Diag(gamma) S0 + Z W,   O = Qe S0 + P W.
+// On the tensor cores everything is transposed so that the 128 value
+// channels are the MMA M dimension (tensor-memory lanes), and S0 enters as
+// bf16(eps * S0)^T:
+//   MMA1  [(Ke S0)^T | (Qe S0)^T] = (eps S0)^T [Kr ; Qr]^T      (N = 64, K = 128)
+//   MMA2  [O^T | S_next^T] += [V^T | -(Ke S0)^T] [P ; Z]^T      (N = 160, K = 2 x 32)
+// The fp32 state lives in tensor memory as the accumulator of MMA2: before
+// each step the scan warpgroup replaces it by gamma * S0^T (fp32, exact
+// decay) and writes the bf16 operand of MMA1.  Everything that does not
+// involve S0 (gate, decays, A_kk, A_qk, T, P, Z) is prepared ahead of time.
 //
-// CTA = one (sequence, head) chain, 416 threads:
-//   warps 0-3   scan warpgroup: issues the inter-chunk MMAs, updates the
-//               state, writes o and hT.
-//   warps 4-7,  two intra warpgroups, alternating 32-token batches: gate,
-//   warps 8-11  decay products, scaled bf16 operands, forward substitution,
-//               W readback; each issues its own intra-chunk MMAs.
-//   warp 12     producer: TMA loads of q, k, v, g (128B swizzle) and beta.
-// Every mbarrier wait is bounded; a wait that runs out raises the device
-// status word, makes the CTA drain its own copies and MMAs, free its tensor
-// memory and return.
+// CTA = one (sequence, head) chain, 512 threads:
+//   warps 0-3   scan warpgroup: one thread per value channel; thread 0
+//               issues the step products and the tile loads of every step.
+//   warps 4-15  three prep warpgroups, taking steps in turn: gate and decay,
+//               scaled operands (in place in the step's tile slot), the
+//               A_kk / A_qk product, forward substitution for T, P, the Z
+//               product, and the bf16 operand [P ; Z] of MMA2.
+// Inside a warpgroup the stages hand over through named barriers that every
+// warp reaches on every step; between warpgroups and with the tensor core,
+// through mbarriers.  Every mbarrier wait is bounded; a wait that runs out
+// raises the device status word, makes the CTA drain its own copies and
+// MMAs, free its tensor memory and return.
 #pragma once
 
 #include "kda_common.cuh"
@@ -54,54 +58,58 @@ namespace prefill {
 
 using namespace kda::sm100;
 
-constexpr int kC = 16;           // chunk length
-constexpr int kD = 128;          // head size (d_k = d_v)
-constexpr int kBatchTok = 32;    // tokens per TMA batch (two chunks)
-constexpr int kRing = 6;         // chunks of scan operands in flight
-constexpr int kThreads = 416;
+constexpr int kTile = 16;          // intra-chunk tile
+constexpr int kStep = 32;          // tokens per state step (two tiles)
+constexpr int kD = 128;            // head size (d_k = d_v)
+constexpr int kBatchTok = kStep;   // rows of one TMA box
+constexpr int kThreads = 512;
+constexpr int kPrep = 3;           // prep warpgroups
+constexpr int kSlots = 4;          // steps whose tiles are resident at once
 
 // ---- shared memory map (offsets from a 1024-aligned base) ----
-// Input slot (32 KB): eight [32 rows][64 ch] 128B-swizzled regions.  The
-// intra warpgroup rewrites k and q in place with K e^{b-m} and Q e^{b-m}.
-constexpr uint32_t OFF_K0 = 0, OFF_Q0 = 4096, OFF_K1 = 8192, OFF_Q1 = 12288;
-constexpr uint32_t OFF_V0 = 16384, OFF_V1 = 20480, OFF_G0 = 24576, OFF_G1 = 28672;
-constexpr uint32_t kSlotBytes = 32768;
-constexpr uint32_t SM_RING = 2 * kSlotBytes;          // kRing x 19 KB
-// Ring slot (one chunk of scan operands):
-constexpr uint32_t R_B1 = 0;         // [-W ; Q e^b] 32 x 128 bf16, K-major SW128 (8 KB)
-constexpr uint32_t R_KHF = 8192;     // (K e^{m-b})^T 128 x 16 fp32, K-major no-swizzle (8 KB):
-                                     // channel rows, 4-token 16-byte cores, LBO 2048, SBO 128
-constexpr uint32_t R_TT = 16384;     // [T ; 0] 32 x 16 bf16, no-swizzle K-major (1 KB)
-constexpr uint32_t R_AQ = 17408;     // causal A_qk 16 x 16 fp32, no-swizzle K-major (1 KB)
-constexpr uint32_t R_DELTA = 18432;  // e^{b_15 - m}, 128 fp32
-constexpr uint32_t R_EPS = 18944;    // e^{m}, 128 fp32
-constexpr uint32_t kRingBytes = 19456;
-// K e^{m-b} of a 32-token batch in bf16 (both chunks, contiguous rows),
-// [32][64] x 2, 128B swizzle: B operand of the A_kk/A_qk MMA.  One per
-// batch of the ring.
-constexpr int kKhRing = kRing / 2;
-constexpr uint32_t SM_KH = SM_RING + kRing * kRingBytes;
-constexpr uint32_t kKhBytes = 8192;
-constexpr uint32_t kSmemBytes = SM_KH + kKhRing * kKhBytes;      // 206848
+// Tile slot of one step: k, q, g, v as [32 rows][64 ch] 128B-swizzled boxes.
+// The gate pass overwrites k, q, g in place with Kr, Qr, Kh; the slot also
+// holds [P ; Z], operand B of MMA2 (160 rows x 32 tokens, K-major, no swizzle).
+constexpr uint32_t SL_K0 = 0, SL_Q0 = 4096, SL_K1 = 8192, SL_Q1 = 12288;
+constexpr uint32_t SL_G0 = 16384, SL_G1 = 20480, SL_V0 = 24576, SL_V1 = 28672;
+constexpr uint32_t SL_B2 = 32768;
+constexpr uint32_t kSlotBytes = 43008;
+// Solve scratch of a prep warpgroup.
+constexpr uint32_t kScRow = 144;      // bytes per row of the fp32 scratch matrix (36 floats)
+constexpr uint32_t SC_AT = 0;         // (Diag(beta) strict_lower(A_kk))^T, fp32 [32][36]
+constexpr uint32_t SC_TB = 4608;      // T bf16, K-major no swizzle (row = column of T): B of Z and P
+constexpr uint32_t SC_AQ = 6656;      // causal(A_qk) bf16, K-major no swizzle: A of the P product
+constexpr uint32_t kScBytes = 8704;
+constexpr uint32_t SM_SLOT = 0;
+constexpr uint32_t SM_SC = SM_SLOT + kSlots * kSlotBytes;
+constexpr uint32_t SM_GAMMA = SM_SC + kPrep * kScBytes;      // kSlots x 128 fp32
+constexpr uint32_t SM_EPS = SM_GAMMA + kSlots * 512;         // kSlots x 128 fp32
+constexpr uint32_t SM_DELTA = SM_EPS + kSlots * 512;         // kPrep x 128 fp32
+// The P product reads 128 rows of its A operand (only the first 32 are
+// causal(A_qk)); the tail pad keeps the other rows inside the allocation.
+constexpr uint32_t kSmemBytes = SM_DELTA + kPrep * 512 + 8192;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
+static_assert(kSlotBytes % 1024 == 0, "slot alignment");
 
 // ---- tensor memory columns ----
-constexpr uint32_t COL_SCR = 0;                  // 2 x 32: per intra warpgroup
-constexpr uint32_t COL_RING = 64;                // kRing x 32: [U | O]^T
-constexpr uint32_t COL_Y = COL_RING + 32 * kRing;    // 128: state accumulator
-constexpr uint32_t COL_SBF = COL_Y + 128;        // 64: bf16 S^T (MMA A operand)
+constexpr uint32_t COL_UP = 0;       // 32: (Ke S0)^T
+constexpr uint32_t COL_O = 32;       // 32: O^T
+constexpr uint32_t COL_S = 64;       // 128: S^T accumulator
+constexpr uint32_t COL_S16 = 192;    // 64: bf16 (eps S)^T, A operand of MMA1
+constexpr uint32_t COL_UN = 256;     // 16: bf16 -(Ke S0)^T, A operand of MMA2
+constexpr uint32_t COL_PREP = 288;   // kPrep x 64: prep accumulators (A_kk | A_qk, then Z | P)
 constexpr uint32_t kTmemCols = 512;
-static_assert(COL_SBF + 64 <= kTmemCols, "tensor memory map overflow");
+static_assert(COL_PREP + 64 * kPrep <= kTmemCols, "tensor memory map overflow");
 
 // A pipeline stage never waits more than microseconds; give up after ~2 s.
 constexpr unsigned long long kWaitLimit = 1ull << 32;
 
 #ifdef KDA_TRACE
 // Stage timestamps (clock64) of the chain run by CTA 0; a profiling build only.
-enum { TR_SCAN_MMA1 = 0, TR_SCAN_MMA1_DONE, TR_SCAN_MMA2, TR_SCAN_MMA2_DONE, TR_SCAN_END,
-       TR_INTRA_FULL, TR_INTRA_P1, TR_INTRA_KQ, TR_INTRA_P2, TR_INTRA_W, TR_INTRA_P3,
-       TR_PROD_ISSUE, TR_SCAN_OUT, TR_SCAN_RF, TR_EVENTS };
-constexpr int kTraceLen = 128;
+enum { TR_SCAN_ISSUE = 0, TR_SCAN_U, TR_SCAN_DONE, TR_SCAN_READY, TR_PREP_FULL, TR_PREP_P1,
+       TR_PREP_A, TR_PREP_T, TR_PREP_Z, TR_PREP_B,
+       TR_S_M1, TR_S_UST, TR_S_BR, TR_S_LD, TR_S_H0, TR_S_H1, TR_S_OLD, TR_EVENTS };
+constexpr int kTraceLen = 256;
 __device__ unsigned long long g_trace[TR_EVENTS][kTraceLen];
 __device__ unsigned long long g_cta_time[1024][3];   // globaltimer start, end, smid
 #define KDA_TR(ev, idx)                                                              \
@@ -113,12 +121,12 @@ __device__ unsigned long long g_cta_time[1024][3];   // globaltimer start, end, 
 #endif
 
 struct Barriers {
-    uint64_t slot_full[2], slot_empty[2];
-    uint64_t intra1[2], kq_done[2], intra2[2], w_done[2];
-    uint64_t ring_full[kRing], ring_empty[kRing];
-    uint64_t mma1_done, mma2_done, sbf_ready;
-    uint64_t drain_scan, drain_intra[2];
-    float beta_s[2][kBatchTok];
+    uint64_t slot_full[kSlots];
+    uint64_t a_done[kPrep], z_done[kPrep], b_ready[kPrep];
+    uint64_t mma1_done, d_done;
+    uint64_t drain_scan, drain_prep[kPrep];
+    float beta_s[kPrep][kStep];
+    int stop[kPrep + 1];             // per-warpgroup exit decision (last: scan)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -222,9 +230,13 @@ __device__ __forceinline__ float rcp(float x) {
     return y;
 }
 
-// decay factor a = exp(-5 sigmoid(g)), via exp2
-__device__ __forceinline__ float decay(float g) {
-    return ex2(-5.0f * kLog2e * rcp(1.0f + ex2(-g * kLog2e)));
+// decay factors a = exp(-5 sigmoid(g)) of a channel pair, via exp2
+__device__ __forceinline__ float2 decay2(float2 g) {
+    const float2 x = fmul2(g, make_float2(-kLog2e, -kLog2e));
+    const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), make_float2(1.f, 1.f));
+    const float2 l = fmul2(make_float2(rcp(den.x), rcp(den.y)),
+                           make_float2(-5.f * kLog2e, -5.f * kLog2e));
+    return make_float2(ex2(l.x), ex2(l.y));
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
@@ -241,57 +253,66 @@ __device__ __forceinline__ void fail(Barriers &bars) {
     raise_error(kErrTimeout);
 }
 
-__device__ __forceinline__ uint4 pack16(const float (&x)[kC]) {
-    uint4 r;
-    r.x = pack_bf16(x[0], x[1]);
-    r.y = pack_bf16(x[2], x[3]);
-    r.z = pack_bf16(x[4], x[5]);
-    r.w = pack_bf16(x[6], x[7]);
-    return r;
+// Barrier among the warps of one warpgroup (id >= 1; 0 is __syncthreads).
+__device__ __forceinline__ void group_sync(int id) {
+    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
 
-// End-of-chunk state pass of the scan warpgroup (one thread = one value
-// channel = one TMEM lane): S = delta * Y, its bf16 copy for the next chunk's
-// MMA, and either Y = eps_next * S for the next chunk or S itself to hT.
-template <bool kNext>
-__device__ __forceinline__ void state_pass(uint32_t tlane, const float4 *dl4, const float4 *ep4,
-                                           float *hdst) {
+// Byte offset of element (row n, k) of a K-major no-swizzle bf16 tile with
+// 32 k per row: 8-row x 16-byte core matrices, LBO 128 (next 8 k), SBO 512
+// (next 8 rows).
+__host__ __device__ __forceinline__ uint32_t core32_off(uint32_t n, uint32_t k) {
+    return (n >> 3) * 512u + (k >> 3) * 128u + (n & 7u) * 16u + (k & 7u) * 2u;
+}
+
+// Gate, decay and scaled operands of one step, in place in its tile slot.
+// Thread (pw, lane) of a prep warpgroup handles rows 16 (pw >> 1) .. + 15
+// and key channels 64 (pw & 1) + 2 lane, + 1.  kFull: all 32 rows are tokens
+// of the sequence (no masking).  Writes eps (first tile) or delta (second).
+template <bool kFull>
+__device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane, int Ls,
+                                          float *eps_out, float *dlt_out) {
+    const int th = pw >> 1, kb = pw & 1, cc = 2 * lane;
+    const int r0 = 16 * th;
+    const uint32_t oK = kb ? SL_K1 : SL_K0, oQ = kb ? SL_Q1 : SL_Q0;
+    const uint32_t oG = kb ? SL_G1 : SL_G0;
+    const float2 one = make_float2(1.f, 1.f);
+    float2 eb[kTile];
+    float2 acc = one;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t y[64];
-        tmem_ld32(tlane + COL_Y + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(y));
-        tmem_ld32(tlane + COL_Y + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(y + 32));
-        tmem_wait_ld();
-        uint32_t sbv[32];
+    for (int rr = 0; rr < kTile; ++rr) {
+        const int r = r0 + rr;
+        const float2 g = bf16x2_to_float2(
+            *reinterpret_cast<const uint32_t *>(slot + oG + sw128_off(r, cc)));
+        const float2 a = decay2(g);
+        acc = fmul2(acc, (kFull || r < Ls) ? a : one);
+        eb[rr] = acc;
+    }
+    // first tile: b - m = log(eb / eb_15); second tile: b - m = log(eb)
+    const float2 tot = eb[kTile - 1];
+    float2 base = one, top = one;
+    if (th == 0) {
+        base = make_float2(rcp(tot.x), rcp(tot.y));
+        top = tot;
+        *reinterpret_cast<float2 *>(eps_out + 64 * kb + cc) = tot;
+    } else {
+        *reinterpret_cast<float2 *>(dlt_out + 64 * kb + cc) = tot;
+    }
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const float4 d = dl4[16 * half + q];
-            float2 s01 = fmul2(make_float2(d.x, d.y),
-                               make_float2(__uint_as_float(y[4 * q]), __uint_as_float(y[4 * q + 1])));
-            float2 s23 = fmul2(make_float2(d.z, d.w),
-                               make_float2(__uint_as_float(y[4 * q + 2]), __uint_as_float(y[4 * q + 3])));
-            sbv[2 * q] = pack_bf16(s01.x, s01.y);
-            sbv[2 * q + 1] = pack_bf16(s23.x, s23.y);
-            if (kNext) {
-                const float4 e = ep4[16 * half + q];
-                s01 = fmul2(make_float2(e.x, e.y), s01);
-                s23 = fmul2(make_float2(e.z, e.w), s23);
-            }
-            y[4 * q] = __float_as_uint(s01.x);
-            y[4 * q + 1] = __float_as_uint(s01.y);
-            y[4 * q + 2] = __float_as_uint(s23.x);
-            y[4 * q + 3] = __float_as_uint(s23.y);
-        }
-        tmem_st16(tlane + COL_SBF + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(sbv));
-        tmem_st16(tlane + COL_SBF + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(sbv + 16));
-        if (kNext) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                tmem_st16(tlane + COL_Y + 64 * half + 16 * q4, *reinterpret_cast<uint32_t(*)[16]>(y + 16 * q4));
-        } else if (hdst) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i) hdst[(size_t)(64 * half + i) * kD] = __uint_as_float(y[i]);
-        }
+    for (int rr = 0; rr < kTile; ++rr) {
+        const int r = r0 + rr;
+        const uint32_t o = sw128_off(r, cc);
+        const bool live = kFull || r < Ls;
+        const uint32_t kraw = *reinterpret_cast<const uint32_t *>(slot + oK + o);
+        const uint32_t qraw = *reinterpret_cast<const uint32_t *>(slot + oQ + o);
+        const float2 kf = bf16x2_to_float2(live ? kraw : 0u);
+        const float2 qf = bf16x2_to_float2(live ? qraw : 0u);
+        const float2 er = fmul2(eb[rr], base);                                  // e^{b-m}
+        const float2 ei = fmul2(top, make_float2(rcp(eb[rr].x), rcp(eb[rr].y)));  // e^{m-b}
+        const float2 kr = fmul2(kf, er), qr = fmul2(qf, er), kh = fmul2(kf, ei);
+        *reinterpret_cast<uint32_t *>(slot + oK + o) = pack_bf16(kr.x, kr.y);
+        *reinterpret_cast<uint32_t *>(slot + oQ + o) = pack_bf16(qr.x, qr.y);
+        *reinterpret_cast<uint32_t *>(slot + oG + o) = pack_bf16(kh.x, kh.y);
     }
 }
 
@@ -322,27 +343,21 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
     const int h = ch.h;
     const int64_t start = ch.start;
     const int L = ch.L;
-    const int nC = (L + kC - 1) / kC;
-    const int nB = (nC + 1) / 2;
+    const int nS = (L + kStep - 1) / kStep;
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars.slot_full[i], 2);
-            mbar_init(&bars.slot_empty[i], 1);
-            mbar_init(&bars.intra1[i], 4);
-            mbar_init(&bars.kq_done[i], 1);
-            mbar_init(&bars.intra2[i], 4);
-            mbar_init(&bars.w_done[i], 1);
-            mbar_init(&bars.drain_intra[i], 1);
-        }
-        for (int i = 0; i < kRing; ++i) {
-            mbar_init(&bars.ring_full[i], 4);
-            mbar_init(&bars.ring_empty[i], 4);
+        for (int i = 0; i < kSlots; ++i) mbar_init(&bars.slot_full[i], 1);
+        for (int i = 0; i < kPrep; ++i) {
+            mbar_init(&bars.a_done[i], 1);
+            mbar_init(&bars.z_done[i], 1);
+            mbar_init(&bars.b_ready[i], 1);
+            mbar_init(&bars.drain_prep[i], 1);
+            bars.stop[i] = 0;
         }
         mbar_init(&bars.mma1_done, 1);
-        mbar_init(&bars.mma2_done, 1);
-        mbar_init(&bars.sbf_ready, 4);
+        mbar_init(&bars.d_done, 1);
         mbar_init(&bars.drain_scan, 1);
+        bars.stop[kPrep] = 0;
         bars.abort_flag = 0;
         fence_mbar_init();
     }
@@ -350,12 +365,6 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         tmem_alloc(&bars.tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    // zero the lower half of every [T ; 0] tile (rows 16..31), once
-    for (int e = tid; e < kRing * 128; e += kThreads) {
-        const int s = e / 128, w = e % 128;
-        reinterpret_cast<uint32_t *>(sm + SM_RING + s * kRingBytes + R_TT + 512)[w] = 0u;
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     __syncthreads();
@@ -363,423 +372,444 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
     const uint32_t tm = bars.tmem_base;
     const uint32_t s_base = smem_u32(sm);
 
-    if (warp == 12) {
-        // ------------------------------------------------ producer
-        int last_use0 = -1, last_use1 = -1;
-        if (nB > 0 && lane == 0) {
-            prefetch_tmap(&map_q);
+    if (warp < 4) {
+        // ================================================ scan warpgroup
+        const int j = tid;                                  // value channel = TMEM lane
+        const uint32_t la = (uint32_t)(32 * warp) << 16;
+        bool issued = false;
+        const float *h0u = ch.h0 ? ch.h0 + j : nullptr;
+        constexpr uint32_t id1 = idesc_bf16(128, 64, false, false);
+        constexpr uint32_t id2 = idesc_bf16(128, 160, false, false);
+        constexpr uint32_t id2v = idesc_bf16(128, 160, true, false);
+
+        int loads = 0;                                      // steps whose tiles were requested
+        auto load_step = [&](int s) {     // k, q, g, v rows of step s -> slot s % kSlots
+            unsigned char *slot = sm + SM_SLOT + (s % kSlots) * kSlotBytes;
+            uint64_t *full = &bars.slot_full[s % kSlots];
+            const int z = (int)(start + (int64_t)kStep * s);
+            mbar_expect_tx(full, ch.v_zero ? 24576u : 32768u);
+            tma_load_3d(slot + SL_K0, &map_k, full, 0, h, z);
+            tma_load_3d(slot + SL_K1, &map_k, full, 64, h, z);
+            tma_load_3d(slot + SL_Q0, &map_q, full, 0, h, z);
+            tma_load_3d(slot + SL_Q1, &map_q, full, 64, h, z);
+            tma_load_3d(slot + SL_G0, &map_g, full, 0, h, z);
+            tma_load_3d(slot + SL_G1, &map_g, full, 64, h, z);
+            if (!ch.v_zero) {
+                tma_load_3d(slot + SL_V0, &map_v, full, 0, h, z);
+                tma_load_3d(slot + SL_V1, &map_v, full, 64, h, z);
+            }
+            ++loads;
+        };
+        auto prefetch_step = [&](int s) {   // warm L2 for a later step
+            const int z = (int)(start + (int64_t)kStep * s);
+            for (int x = 0; x < 128; x += 64) {
+                tma_prefetch_3d(&map_k, x, h, z);
+                tma_prefetch_3d(&map_q, x, h, z);
+                tma_prefetch_3d(&map_g, x, h, z);
+                if (!ch.v_zero) tma_prefetch_3d(&map_v, x, h, z);
+            }
+        };
+        // tile loads come from lane 0 of warp 1 and L2 prefetches from lane 0
+        // of warp 2: both are idle while MMA1 runs, off the issuing thread
+        const bool loader = tid == 32, prefetcher = tid == 64;
+        if (loader && nS > 0) {
             prefetch_tmap(&map_k);
-            prefetch_tmap(&map_v);
+            prefetch_tmap(&map_q);
             prefetch_tmap(&map_g);
+            prefetch_tmap(&map_v);
+            for (int s = 0; s < kSlots && s < nS; ++s) load_step(s);
         }
-        for (int b = 0; b < nB; ++b) {
-            const int slot = b & 1, use = b >> 1;
-            if (use > 0 && !warp_wait(&bars.slot_empty[slot], (use - 1) & 1, abortp)) {
-                fail(bars);
-                break;
-            }
-            uint64_t *full = &bars.slot_full[slot];
-            if (lane == 0) {
-                KDA_TR(TR_PROD_ISSUE, b);
-                unsigned char *sb = sm + slot * kSlotBytes;
-                mbar_expect_tx(full, ch.v_zero ? kSlotBytes - 8192 : kSlotBytes);
-                const int z = (int)(start + (int64_t)b * kBatchTok);
-                tma_load_3d(sb + OFF_K0, &map_k, full, 0, h, z);
-                tma_load_3d(sb + OFF_K1, &map_k, full, 64, h, z);
-                tma_load_3d(sb + OFF_Q0, &map_q, full, 0, h, z);
-                tma_load_3d(sb + OFF_Q1, &map_q, full, 64, h, z);
-                if (!ch.v_zero) {
-                    tma_load_3d(sb + OFF_V0, &map_v, full, 0, h, z);
-                    tma_load_3d(sb + OFF_V1, &map_v, full, 64, h, z);
-                }
-                tma_load_3d(sb + OFF_G0, &map_g, full, 0, h, z);
-                tma_load_3d(sb + OFF_G1, &map_g, full, 64, h, z);
-            }
-            const int tok = b * kBatchTok + lane;
-            bars.beta_s[slot][lane] =
-                tok < L ? __bfloat162float(p.beta[(size_t)(start + tok) * p.H + h]) : 0.f;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full);
-            if (slot == 0) last_use0 = use; else last_use1 = use;
-        }
-        // drain: every issued load must land before the CTA exits
-        if (lane == 0) {
-            if (last_use0 >= 0) mbar_wait(&bars.slot_full[0], last_use0 & 1, abortp, kWaitLimit);
-            if (last_use1 >= 0) mbar_wait(&bars.slot_full[1], last_use1 & 1, abortp, kWaitLimit);
-        }
-    } else if (warp >= 4) {
-        // ------------------------------------------------ intra warpgroups
-        const int wg = (warp - 4) >> 2;           // 0 or 1: batches b = wg, wg + 2, ...
-        const int it = tid - 128 - 128 * wg;
-        const int iw = it >> 5;                   // TMEM lane quarter
-        const int j = iw >> 1;                    // chunk of the batch (pass 1)
-        const int kb = iw & 1;                    // 64-channel half (pass 1)
-        const int cc = 2 * lane;                  // column pair inside the half
-        const uint32_t offK = kb ? OFF_K1 : OFF_K0, offQ = kb ? OFF_Q1 : OFF_Q0;
-        const uint32_t offV = kb ? OFF_V1 : OFF_V0, offG = kb ? OFF_G1 : OFF_G0;
-        const uint32_t col_scr = COL_SCR + 32 * wg;
-        const int slot = wg;
-        unsigned char *sb = sm + slot * kSlotBytes;
-        const uint32_t sb_u = s_base + slot * kSlotBytes;
-        bool ok = true, issued = false;
-        for (int kk_b = 0;; ++kk_b) {
-            const int b = wg + 2 * kk_b;
-            if (b >= nB) break;
-            const uint32_t par = kk_b & 1;
-            // ring slots for the two chunks must be free, inputs landed
-            for (int jj = 0; jj < 2 && ok; ++jj) {
-                const int cj = 2 * b + jj;
-                if (cj < nC && cj >= kRing)
-                    ok = warp_wait(&bars.ring_empty[cj % kRing], ((cj / kRing) - 1) & 1, abortp);
-            }
-            if (ok) ok = warp_wait(&bars.slot_full[slot], par, abortp);
-            if (!ok) { fail(bars); break; }
-            if (it == 0) KDA_TR(TR_INTRA_FULL, b);
-
-            // ---------------- pass 1: gate, decay, scaled operands
-            {
-                const int cj = 2 * b + j;
-                const bool chunk_valid = cj < nC;
-                const int Lj = chunk_valid ? min(kC, L - kC * cj) : 0;
-                unsigned char *ring = sm + SM_RING + (cj % kRing) * kRingBytes;
-                unsigned char *khb = sm + SM_KH + (b % kKhRing) * kKhBytes;
-                float2 eb[kC];                   // e^{b_r} as running products
-                float2 acc = make_float2(1.f, 1.f);
-                const float2 kNegLog2e = make_float2(-kLog2e, -kLog2e);
-                const float2 kNeg5Log2e = make_float2(-5.f * kLog2e, -5.f * kLog2e);
-                const float2 kOne = make_float2(1.f, 1.f);
-#pragma unroll
-                for (int r = 0; r < kC; ++r) {
-                    const uint32_t o = sw128_off(16 * j + r, cc);
-                    const float2 g = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(sb + offG + o));
-                    const float2 x = fmul2(g, kNegLog2e);
-                    const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), kOne);
-                    const float2 l = fmul2(make_float2(rcp(den.x), rcp(den.y)), kNeg5Log2e);
-                    const float2 a = make_float2(ex2(l.x), ex2(l.y));
-                    acc = fmul2(acc, (r < Lj) ? a : kOne);
-                    eb[r] = acc;
-                }
-                const float2 em = eb[7];                                   // e^{m}
-                const float2 im = make_float2(rcp(em.x), rcp(em.y));       // e^{-m}
-                if (chunk_valid) {
-                    float *dl = reinterpret_cast<float *>(ring + R_DELTA);
-                    float *ep = reinterpret_cast<float *>(ring + R_EPS);
-                    *reinterpret_cast<float2 *>(dl + 64 * kb + cc) = fmul2(eb[kC - 1], im);
-                    *reinterpret_cast<float2 *>(ep + 64 * kb + cc) = em;
-                }
-                const int chn = 64 * kb + cc;             // first of this thread's two channels
-                // (channel, token) of the fp32 K-hat tile:
-                // token/4 * 2048 + channel/8 * 128 + channel%8 * 16 + token%4 * 4
-                const uint32_t khf_off = R_KHF + (chn >> 3) * 128 + (chn & 7) * 16;
-                float4 kq0 = make_float4(0.f, 0.f, 0.f, 0.f), kq1 = kq0;
-#pragma unroll
-                for (int r = 0; r < kC; ++r) {
-                    const uint32_t o = sw128_off(16 * j + r, cc);
-                    const bool live = r < Lj;
-                    const uint32_t kraw = *reinterpret_cast<const uint32_t *>(sb + offK + o);
-                    const uint32_t qraw = *reinterpret_cast<const uint32_t *>(sb + offQ + o);
-                    const float2 kf = bf16x2_to_float2(live ? kraw : 0u);
-                    const float2 qf = bf16x2_to_float2(live ? qraw : 0u);
-                    const float2 er = fmul2(eb[r], im);                    // e^{b-m}
-                    const float2 ei = make_float2(rcp(er.x), rcp(er.y));   // e^{m-b}
-                    const float2 kr = fmul2(kf, er), qr = fmul2(qf, er);
-                    const float2 kh = fmul2(kf, ei), qa = fmul2(qf, eb[r]);
-                    *reinterpret_cast<uint32_t *>(sb + offK + o) = pack_bf16(kr.x, kr.y);
-                    *reinterpret_cast<uint32_t *>(sb + offQ + o) = pack_bf16(qr.x, qr.y);
-                    *reinterpret_cast<uint32_t *>(khb + kb * 4096 + sw128_off(16 * j + r, cc)) =
-                        pack_bf16(kh.x, kh.y);
-                    if (chunk_valid)
-                        *reinterpret_cast<uint32_t *>(ring + R_B1 + kb * 4096 + sw128_off(16 + r, cc)) =
-                            pack_bf16(qa.x, qa.y);
-                    // four consecutive tokens of each of the two channels -> one 16-byte core row
-                    if ((r & 3) == 0) { kq0.x = kh.x; kq1.x = kh.y; }
-                    if ((r & 3) == 1) { kq0.y = kh.x; kq1.y = kh.y; }
-                    if ((r & 3) == 2) { kq0.z = kh.x; kq1.z = kh.y; }
-                    if ((r & 3) == 3) {
-                        kq0.w = kh.x; kq1.w = kh.y;
-                        if (chunk_valid) {
-                            *reinterpret_cast<float4 *>(ring + khf_off + (r >> 2) * 2048) = kq0;
-                            *reinterpret_cast<float4 *>(ring + khf_off + (r >> 2) * 2048 + 16) = kq1;
-                        }
-                    }
-                }
-                // rows past the end of the sequence (every row when v is
-                // treated as zero): V must be exactly zero
-                const int vz = ch.v_zero ? 0 : Lj;
-                if (vz < kC)
-                    for (int r = vz; r < kC; ++r)
-                        *reinterpret_cast<uint32_t *>(sb + offV + sw128_off(16 * j + r, cc)) = 0u;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.intra1[wg]);
-            if (it == 0) KDA_TR(TR_INTRA_P1, b);
-
-            // ---------------- MMA: A_kk and A_qk rows of both chunks
-            if (it == 0) {
-                if (!mbar_wait(&bars.intra1[wg], par, abortp, kWaitLimit)) { fail(bars); ok = false; }
-                else {
-                    tc_fence_after();
-                    constexpr uint32_t id = idesc_bf16(128, 32, false, false);
-                    const uint32_t kh = s_base + SM_KH + (b % kKhRing) * kKhBytes;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t a = sdesc(sb_u + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-                        const uint64_t bd = sdesc(kh + (kk >> 2) * 4096 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-                        mma_ss(tm + col_scr, a, bd, id, kk > 0);
-                    }
-                    tc_commit(&bars.kq_done[wg]);
-                    issued = true;
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-
-            // ---------------- pass 2: forward substitution (warp 0), causal A_qk (warp 1)
-            if (iw < 2) {
-                if (!warp_wait(&bars.kq_done[wg], par, abortp)) { fail(bars); ok = false; break; }
-                if (it == 0) KDA_TR(TR_INTRA_KQ, b);
-                tc_fence_after();
-                uint32_t d[32];
-                tmem_ld32(tm + ((uint32_t)(32 * iw) << 16) + col_scr, d);
-                tmem_wait_ld();
-                const int jj = lane >> 4, r = lane & 15;
-                const int cj = 2 * b + jj;
-                unsigned char *ring = sm + SM_RING + (cj % kRing) * kRingBytes;
-                float X[kC];
-                if (iw == 0) {
-                    const float beta_l = bars.beta_s[slot][lane];
-                    float A[kC];
-#pragma unroll
-                    for (int i = 0; i < kC; ++i) {
-                        const float a = __uint_as_float(jj ? d[16 + i] : d[i]);
-                        A[i] = (i < r) ? beta_l * a : 0.f;
-                        X[i] = (i == r) ? beta_l : 0.f;
-                    }
-                    // row r of T = (I + A)^-1 Diag(beta): rows are finished in order
-#pragma unroll
-                    for (int i = 0; i < kC - 1; ++i) {
-#pragma unroll
-                        for (int col = 0; col <= i; ++col) {
-                            const float t = __shfl_sync(0xffffffffu, X[col], i, 16);
-                            if (r > i) X[col] = fmaf(-A[i], t, X[col]);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < kC; ++i) {
-                        const float a = __uint_as_float(jj ? d[16 + i] : d[i]);
-                        X[i] = (i <= r) ? a : 0.f;
-                    }
-                }
-                if (cj < nC) {
-                    if (iw == 0) {   // T in bf16 (B operand of the W / U_v MMAs)
-                        uint4 lo, hi;
-                        lo.x = pack_bf16(X[0], X[1]);   lo.y = pack_bf16(X[2], X[3]);
-                        lo.z = pack_bf16(X[4], X[5]);   lo.w = pack_bf16(X[6], X[7]);
-                        hi.x = pack_bf16(X[8], X[9]);   hi.y = pack_bf16(X[10], X[11]);
-                        hi.z = pack_bf16(X[12], X[13]); hi.w = pack_bf16(X[14], X[15]);
-                        *reinterpret_cast<uint4 *>(ring + R_TT + core16_off(r, 0)) = lo;
-                        *reinterpret_cast<uint4 *>(ring + R_TT + core16_off(r, 8)) = hi;
-                    } else {         // causal A_qk in fp32 (B operand of the tf32 MMA)
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4)
-                            *reinterpret_cast<float4 *>(ring + R_AQ + core16_off32(r, 4 * k4)) =
-                                make_float4(X[4 * k4], X[4 * k4 + 1], X[4 * k4 + 2], X[4 * k4 + 3]);
-                    }
-                }
-                fence_proxy_async_smem();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.intra2[wg]);
-            if (it == 0) KDA_TR(TR_INTRA_P2, b);
-
-            // ---------------- MMA: W^T (unscaled) and [U_v | 0]^T per chunk
-            if (it == 0) {
-                if (!mbar_wait(&bars.intra2[wg], par, abortp, kWaitLimit)) { fail(bars); ok = false; }
-                else {
-                    tc_fence_after();
-                    constexpr uint32_t idw = idesc_bf16(128, 16, true, false);
-                    constexpr uint32_t idu = idesc_bf16(128, 32, true, false);
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int cj = 2 * b + jj;
-                        if (cj >= nC) break;
-                        const uint32_t ring_u = s_base + SM_RING + (cj % kRing) * kRingBytes;
-                        const uint64_t tdesc = sdesc(ring_u + R_TT, 128, 256, kLayoutNone);
-                        mma_ss(tm + col_scr + 16 * jj,
-                               sdesc(sb_u + OFF_K0 + 2048 * jj, OFF_K1 - OFF_K0, 1024, kLayoutSW128),
-                               tdesc, idw, 0);
-                        mma_ss(tm + COL_RING + 32 * (cj % kRing),
-                               sdesc(sb_u + OFF_V0 + 2048 * jj, OFF_V1 - OFF_V0, 1024, kLayoutSW128),
-                               tdesc, idu, 0);
-                    }
-                    tc_commit(&bars.w_done[wg]);
-                    tc_commit(&bars.slot_empty[slot]);
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-
-            // ---------------- pass 3: -W = -(W^T * eps)^T rows of the B1 tiles
-            if (!warp_wait(&bars.w_done[wg], par, abortp)) { fail(bars); ok = false; break; }
-            if (it == 0) KDA_TR(TR_INTRA_W, b);
-            tc_fence_after();
-            {
-                const int c = 32 * iw + lane;            // key channel (TMEM lane)
-                const int wkb = c >> 6, wcol = c & 63;
-                for (int jj = 0; jj < 2; ++jj) {
-                    const int cj = 2 * b + jj;
-                    if (cj >= nC) break;
-                    uint32_t w[16];
-                    tmem_ld16(tm + ((uint32_t)(32 * iw) << 16) + col_scr + 16 * jj, w);
-                    tmem_wait_ld();
-                    unsigned char *ring = sm + SM_RING + (cj % kRing) * kRingBytes;
-                    const float neps = -reinterpret_cast<const float *>(ring + R_EPS)[c];
-#pragma unroll
-                    for (int r = 0; r < kC; ++r)
-                        *reinterpret_cast<__nv_bfloat16 *>(ring + R_B1 + wkb * 4096 + sw128_off(r, wcol)) =
-                            __float2bfloat16_rn(neps * __uint_as_float(w[r]));
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                for (int jj = 0; jj < 2; ++jj)
-                    if (2 * b + jj < nC) mbar_arrive(&bars.ring_full[(2 * b + jj) % kRing]);
-            if (it == 0) KDA_TR(TR_INTRA_P3, b);
-        }
-        // drain this warpgroup's MMAs before the CTA frees tensor memory
-        if (it == 0 && issued) {
-            tc_commit(&bars.drain_intra[wg]);
-            mbar_wait(&bars.drain_intra[wg], 0, abortp, kWaitLimit);
-        }
-    } else {
-        // ------------------------------------------------ scan warpgroup
-        const int jv = tid;                               // value channel = TMEM lane
-        const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
-        bool ok = true, issued = false;
-        const float *h0u = ch.h0 ? ch.h0 + jv : nullptr;
-        if (nC > 0) {
-            // initial state: bf16 copy for the first MMA, eps_0 * S0 into Y
-            ok = warp_wait(&bars.ring_full[0], 0, abortp);
-            if (!ok) fail(bars);
-            else {
-                tc_fence_after();
-                const float *ep = reinterpret_cast<const float *>(sm + SM_RING + R_EPS);
-#pragma unroll
+        if (prefetcher)
+            for (int s = kSlots; s < 2 * kSlots && s < nS; ++s) prefetch_step(s);
+        bool alive = nS > 0;
+        if (alive) {
+            // initial state: gamma_0 * S0 (fp32) and bf16(eps_0 * S0)
+            if (warp_wait(&bars.b_ready[0], 0, abortp)) {
+                const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA);
+                const float4 *e4 = reinterpret_cast<const float4 *>(sm + SM_EPS);
+#pragma unroll 1
                 for (int part = 0; part < 4; ++part) {
                     float s0[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        s0[i] = h0u ? h0u[(size_t)(32 * part + i) * kD]
-                                    : ((ch.h0_identity && 32 * part + i == jv) ? 1.f : 0.f);
-                    uint32_t sb16[16], y0[16], y1[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        sb16[i] = pack_bf16(s0[2 * i], s0[2 * i + 1]);
-                        y0[i] = __float_as_uint(ep[32 * part + i] * s0[i]);
-                        y1[i] = __float_as_uint(ep[32 * part + 16 + i] * s0[16 + i]);
+                    for (int i = 0; i < 32; ++i) {
+                        const int row = 32 * part + i;
+                        s0[i] = h0u ? h0u[(size_t)row * kD]
+                                    : ((ch.h0_identity && row == j) ? 1.f : 0.f);
                     }
-                    tmem_st16(tm + lane_addr + COL_SBF + 16 * part, sb16);
-                    tmem_st16(tm + lane_addr + COL_Y + 32 * part, y0);
-                    tmem_st16(tm + lane_addr + COL_Y + 32 * part + 16, y1);
+                    uint32_t sb[16], y[32];
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 gm = g4[8 * part + q4], ep = e4[8 * part + q4];
+                        sb[2 * q4] = pack_bf16(ep.x * s0[4 * q4], ep.y * s0[4 * q4 + 1]);
+                        sb[2 * q4 + 1] = pack_bf16(ep.z * s0[4 * q4 + 2], ep.w * s0[4 * q4 + 3]);
+                        y[4 * q4] = __float_as_uint(gm.x * s0[4 * q4]);
+                        y[4 * q4 + 1] = __float_as_uint(gm.y * s0[4 * q4 + 1]);
+                        y[4 * q4 + 2] = __float_as_uint(gm.z * s0[4 * q4 + 2]);
+                        y[4 * q4 + 3] = __float_as_uint(gm.w * s0[4 * q4 + 3]);
+                    }
+                    tmem_st16(tm + la + COL_S16 + 16 * part, sb);
+                    tmem_st16(tm + la + COL_S + 32 * part, *reinterpret_cast<uint32_t(*)[16]>(y));
+                    tmem_st16(tm + la + COL_S + 32 * part + 16, *reinterpret_cast<uint32_t(*)[16]>(y + 16));
                 }
                 tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.sbf_ready);
+            } else {
+                fail(bars);
             }
+            tc_fence_before();
+            if (tid == 0) bars.stop[kPrep] = *abortp;
+            group_sync(1);
+            alive = bars.stop[kPrep] == 0;
         } else if (ch.hT) {
-            float *dst = ch.hT + jv;
-            for (int c = 0; c < kD; ++c)
-                dst[(size_t)c * kD] = h0u ? h0u[(size_t)c * kD] : ((ch.h0_identity && c == jv) ? 1.f : 0.f);
+            float *dst = ch.hT + j;
+            for (int row = 0; row < kD; ++row)
+                dst[(size_t)row * kD] = h0u ? h0u[(size_t)row * kD]
+                                            : ((ch.h0_identity && row == j) ? 1.f : 0.f);
         }
 
-        for (int c = 0; c < nC && ok; ++c) {
-            const int rs = c % kRing;
-            const uint32_t ring_u = s_base + SM_RING + rs * kRingBytes;
-            const unsigned char *ring = sm + SM_RING + rs * kRingBytes;
-            const uint32_t colU = COL_RING + 32 * rs;
-            // MMA1: [U | O]^T += S^T [-W ; Q e^b]^T  (bf16); then, once it has
-            // landed, MMA2 reads U^T straight from tensor memory as tf32:
-            // O^T += U^T causal(A_qk)^T ;  Y += U^T Kh
-            if (tid == 0) {
-                ok = mbar_wait(&bars.ring_full[rs], (c / kRing) & 1, abortp, kWaitLimit) &&
-                     mbar_wait(&bars.sbf_ready, c & 1, abortp, kWaitLimit);
-                if (ok) {
-                    KDA_TR(TR_SCAN_MMA1, c);
-                    tc_fence_after();
-                    constexpr uint32_t id = idesc_bf16(128, 32, false, false);
-                    const uint64_t b0 = sdesc(ring_u + R_B1, 16, 1024, kLayoutSW128);
+        uint32_t ov[32];                // outputs of the previous step, stored after the next MMA1 issue
+        int o_step = -1;
+        auto store_o = [&]() {
+            if (o_step < 0 || !ch.write_o) return;
+            const int Lc = L - kStep * o_step;
+            __nv_bfloat16 *dst = p.o + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
+            const size_t step = (size_t)p.H * kD;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tm + colU, tm + COL_SBF + 8 * kk,
-                               b0 + (uint64_t)(((kk >> 2) * 4096 + (kk & 3) * 32) >> 4), id, 1);
-                    tc_commit(&bars.mma1_done);
-                    issued = true;
-                    ok = mbar_wait(&bars.mma1_done, c & 1, abortp, kWaitLimit);
-                }
-                if (ok) {
-                    KDA_TR(TR_SCAN_MMA2, c);
-                    tc_fence_after();
-                    constexpr uint32_t ido = idesc_tf32(128, 16, false, false);
-                    constexpr uint32_t idy = idesc_tf32(128, 128, false, false);
-                    const uint64_t aq = sdesc(ring_u + R_AQ, 128, 512, kLayoutNone);
-                    const uint64_t kh = sdesc(ring_u + R_KHF, 2048, 128, kLayoutNone);
+            for (int r = 0; r < kStep; ++r)
+                if (r < Lc) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov[r]));
+            o_step = -1;
+        };
+        for (int c = 0; alive && c < nS; ++c) {
+            const int sl = c % kSlots;
+            const uint32_t slot_u = s_base + SM_SLOT + sl * kSlotBytes;
+            // ---- MMA1: [(Ke S)^T | (Qe S)^T] = bf16(eps S)^T [Kr ; Qr]^T, then the v part of MMA2
+            if (tid == 0 && !*abortp) {
+                KDA_TR(TR_SCAN_ISSUE, c);
+                tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        mma_ts_tf32(tm + colU + 16, tm + colU + 8 * ks, aq + (uint64_t)((256 * ks) >> 4), ido, 1);
-                        mma_ts_tf32(tm + COL_Y, tm + colU + 8 * ks, kh + (uint64_t)((4096 * ks) >> 4), idy, 1);
-                    }
-                    tc_commit(&bars.mma2_done);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tm + COL_UP, tm + COL_S16 + 8 * kk,
+                           sdesc(slot_u + (kk >> 2) * SL_K1 + (kk & 3) * 32, 16, 1024, kLayoutSW128),
+                           id1, kk > 0);
+                tc_commit(&bars.mma1_done);
+                if (!ch.v_zero) {
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        mma_ss(tm + COL_O, sdesc(slot_u + SL_V0 + 2048 * kk, SL_V1 - SL_V0, 1024, kLayoutSW128),
+                               sdesc(slot_u + SL_B2 + 256 * kk, 128, 512, kLayoutNone), id2v, 1);
                 }
-                if (!ok) fail(bars);
+                issued = true;
             }
-            const bool has_next = c + 1 < nC;
-            if (has_next && !warp_wait(&bars.ring_full[(c + 1) % kRing], ((c + 1) / kRing) & 1, abortp)) {
-                fail(bars); ok = false; break;
+            // the slot of step c - 1 was freed by its completed products:
+            // request step c - 1 + kSlots (overlaps the MMA1 round trip)
+            if (loader && c >= 1 && c - 1 + kSlots < nS && !*abortp) load_step(c - 1 + kSlots);
+            if (prefetcher && c >= 1 && c - 1 + 2 * kSlots < nS) prefetch_step(c - 1 + 2 * kSlots);
+            store_o();
+            // ---- -(Ke S)^T in bf16: A operand of the second half of MMA2
+            if (warp_wait(&bars.mma1_done, c & 1, abortp)) {
+                if (tid == 0) KDA_TR(TR_S_M1, c);
+                tc_fence_after();
+                uint32_t u[32], un[16];
+                tmem_ld32(tm + la + COL_UP, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int w = 0; w < 16; ++w)
+                    un[w] = pack_bf16(-__uint_as_float(u[2 * w]), -__uint_as_float(u[2 * w + 1]));
+                tmem_st16(tm + la + COL_UN, un);
+                tmem_wait_st();
+                if (tid == 0) KDA_TR(TR_S_UST, c);
+            } else {
+                fail(bars);
             }
-            if (!warp_wait(&bars.mma2_done, c & 1, abortp)) { fail(bars); ok = false; break; }
-            if (tid == 0) KDA_TR(TR_SCAN_MMA2_DONE, c);
-            tc_fence_after();
-            // this chunk's output (the tensor pipe is idle for this warpgroup now)
-            uint32_t ov[16];
-            tmem_ld16(tm + lane_addr + colU + 16, ov);
-            // S = delta * Y  ->  bf16 copy;  Y = eps_next * S  (or hT at the end)
-            {
-                const float4 *dl4 = reinterpret_cast<const float4 *>(ring + R_DELTA);
-                if (has_next) {
-                    const float4 *ep4 = reinterpret_cast<const float4 *>(
-                        sm + SM_RING + ((c + 1) % kRing) * kRingBytes + R_EPS);
-                    state_pass<true>(tm + lane_addr, dl4, ep4, nullptr);
-                } else {
-                    float *hdst = ch.hT ? ch.hT + jv : nullptr;
-                    state_pass<false>(tm + lane_addr, dl4, nullptr, hdst);
-                }
-            }
-            tmem_wait_st();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars.sbf_ready);
-                mbar_arrive(&bars.ring_empty[rs]);
-            }
-            if (tid == 0) KDA_TR(TR_SCAN_END, c);
-            if (ch.write_o) {
-                const int Lc = min(kC, L - kC * c);
-                __nv_bfloat16 *dst = p.o + ((size_t)(start + kC * c) * p.H + h) * kD + jv;
-                const size_t step = (size_t)p.H * kD;
+            group_sync(1);
+            if (tid == 0 && !*abortp) {
+                KDA_TR(TR_SCAN_U, c);
+                tc_fence_after();
 #pragma unroll
-                for (int r = 0; r < kC; ++r)
-                    if (r < Lc) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov[r]));
+                for (int kk = 0; kk < 2; ++kk)
+                    mma_ts(tm + COL_O, tm + COL_UN + 8 * kk,
+                           sdesc(slot_u + SL_B2 + 256 * kk, 128, 512, kLayoutNone), id2, 1);
+                tc_commit(&bars.d_done);
             }
+            // ---- step done: outputs, next step's operands (or the final state)
+            if (warp_wait(&bars.d_done, c & 1, abortp)) {
+                tc_fence_after();
+                if (tid == 0) KDA_TR(TR_SCAN_DONE, c);
+                const bool has_next = c + 1 < nS;
+                bool ready = true;
+                if (has_next) ready = warp_wait(&bars.b_ready[(c + 1) % kPrep], ((c + 1) / kPrep) & 1, abortp);
+                if (!ready) fail(bars);
+                if (tid == 0) KDA_TR(TR_S_BR, c);
+                const int sn = (c + 1) % kSlots;
+                const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA + sn * 512);
+                const float4 *e4 = reinterpret_cast<const float4 *>(sm + SM_EPS + sn * 512);
+#pragma unroll 1
+                for (int qt = 0; qt < 4 && ready; ++qt) {       // 32 key channels at a time
+                    uint32_t sv[32];
+                    tmem_ld32(tm + la + COL_S + 32 * qt, sv);
+                    tmem_wait_ld();
+                    if (tid == 0 && qt == 0) KDA_TR(TR_S_LD, c);
+                    if (has_next) {
+                        uint32_t sb[16];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 gm = g4[8 * qt + q4], ep = e4[8 * qt + q4];
+                            uint32_t *y = sv + 4 * q4;
+                            const float2 s01 = make_float2(__uint_as_float(y[0]), __uint_as_float(y[1]));
+                            const float2 s23 = make_float2(__uint_as_float(y[2]), __uint_as_float(y[3]));
+                            const float2 e01 = fmul2(make_float2(ep.x, ep.y), s01);
+                            const float2 e23 = fmul2(make_float2(ep.z, ep.w), s23);
+                            sb[2 * q4] = pack_bf16(e01.x, e01.y);
+                            sb[2 * q4 + 1] = pack_bf16(e23.x, e23.y);
+                            const float2 g01 = fmul2(make_float2(gm.x, gm.y), s01);
+                            const float2 g23 = fmul2(make_float2(gm.z, gm.w), s23);
+                            y[0] = __float_as_uint(g01.x);
+                            y[1] = __float_as_uint(g01.y);
+                            y[2] = __float_as_uint(g23.x);
+                            y[3] = __float_as_uint(g23.y);
+                        }
+                        tmem_st16(tm + la + COL_S16 + 16 * qt, sb);
+                        tmem_st16(tm + la + COL_S + 32 * qt, *reinterpret_cast<uint32_t(*)[16]>(sv));
+                        tmem_st16(tm + la + COL_S + 32 * qt + 16, *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
+                        if (tid == 0) KDA_TR(qt == 1 ? TR_S_H0 : TR_S_H1, c);
+                    } else if (ch.hT) {
+                        float *dst = ch.hT + (size_t)(32 * qt) * kD + j;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) dst[(size_t)i * kD] = __uint_as_float(sv[i]);
+                    }
+                }
+                tmem_ld32(tm + la + COL_O, ov);
+                tmem_wait_ld();
+                if (tid == 0) KDA_TR(TR_S_OLD, c);
+                if (ready) o_step = c;
+                tmem_wait_st();
+                tc_fence_before();
+                if (tid == 0) bars.stop[kPrep] = *abortp;
+                group_sync(1);
+                if (tid == 0) KDA_TR(TR_SCAN_READY, c);
+            } else {
+                fail(bars);
+                tc_fence_before();
+                if (tid == 0) bars.stop[kPrep] = 1;
+                group_sync(1);
+            }
+            alive = bars.stop[kPrep] == 0;
         }
+        store_o();                          // outputs of the last step
         if (tid == 0 && issued) {
             tc_commit(&bars.drain_scan);
-            mbar_wait(&bars.drain_scan, 0, abortp, kWaitLimit);
+            mbar_wait_drain(&bars.drain_scan, 0, kWaitLimit);
         }
+        if (loader) {
+            // every requested tile must have landed before the CTA exits
+            for (int s = loads - kSlots < 0 ? 0 : loads - kSlots; s < loads; ++s)
+                mbar_wait_drain(&bars.slot_full[s % kSlots], (s / kSlots) & 1, kWaitLimit);
+        }
+    } else {
+        // ================================================ prep warpgroups
+        const int pg = (warp - 4) >> 2;                 // steps pg, pg + kPrep, ...
+        const int pw = warp & 3;                        // TMEM lane quarter
+        const int pt = tid - 128 - 128 * pg;
+        const int bar_id = 2 + pg;
+        // serial roles on different SM sub-partitions (warp w runs on w % 4;
+        // the scan issuer is warp 0)
+        const int iss_w = 1 + (pg + 1) % 3;             // 2, 3, 1
+        const int solve_w = 1 + pg;                     // 1, 2, 3
+        const bool iss = pw == iss_w && lane == 0;
+        unsigned char *scr = sm + SM_SC + pg * kScBytes;
+        const uint32_t scr_u = s_base + SM_SC + pg * kScBytes;
+        float *dlt = reinterpret_cast<float *>(sm + SM_DELTA + pg * 512);
+        const uint32_t tP = tm + COL_PREP + 64 * pg;
+        const uint32_t tPl = tP + ((uint32_t)(32 * pw) << 16);
+        bool issued = false;
+        constexpr uint32_t idA = idesc_bf16(128, 32, false, false);
+        constexpr uint32_t idZ = idesc_bf16(128, 32, true, false);
+
+        for (int s = pg, u = 0; s < nS; s += kPrep, ++u) {
+            const int sl = s % kSlots;
+            unsigned char *slot = sm + SM_SLOT + sl * kSlotBytes;
+            const uint32_t slot_u = s_base + SM_SLOT + sl * kSlotBytes;
+            const int Ls = min(kStep, L - kStep * s);
+            const uint32_t par = u & 1;
+            if (pw == 0) {
+                const int64_t tok = start + (int64_t)kStep * s + lane;
+                bars.beta_s[pg][lane] =
+                    lane < Ls ? __bfloat162float(p.beta[(size_t)tok * p.H + h]) : 0.f;
+            }
+            bool ok = warp_wait(&bars.slot_full[sl], (s / kSlots) & 1, abortp);
+            if (!ok) fail(bars);
+            if (ok && pt == 0) KDA_TR(TR_PREP_FULL, s);
+
+            // ---------------- gate, decay and scaled operands (in place)
+            if (ok) {
+                float *eps_out = reinterpret_cast<float *>(sm + SM_EPS + sl * 512);
+                if (Ls == kStep) gate_pass<true>(slot, pw, lane, Ls, eps_out, dlt);
+                else gate_pass<false>(slot, pw, lane, Ls, eps_out, dlt);
+            }
+            fence_proxy_async_smem();
+            group_sync(bar_id);                                             // operands written
+
+            // ---------------- A_kk (TMEM lanes 0-31) and A_qk (lanes 32-63)
+            if (iss && !*abortp) {
+                KDA_TR(TR_PREP_P1, s);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = sdesc(slot_u + (kk >> 2) * SL_K1 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
+                    const uint64_t b = sdesc(slot_u + SL_G0 + (kk >> 2) * (SL_G1 - SL_G0) + (kk & 3) * 32,
+                                             16, 1024, kLayoutSW128);
+                    mma_ss(tP, a, b, idA, kk > 0);
+                }
+                tc_commit(&bars.a_done[pg]);
+                issued = true;
+            }
+            if (pw >= 2) {
+                // step decay gamma = eps * delta, for the scan warpgroup
+                if (ok) {
+                    const int c2 = 2 * (pt - 64);
+                    const float2 e2 = *reinterpret_cast<const float2 *>(sm + SM_EPS + sl * 512 + 4 * c2);
+                    const float2 d2 = *reinterpret_cast<const float2 *>(dlt + c2);
+                    *reinterpret_cast<float2 *>(sm + SM_GAMMA + sl * 512 + 4 * c2) = fmul2(e2, d2);
+                }
+            } else {
+                // warp 0: (Diag(beta) strict_lower(A_kk))^T; warp 1: causal(A_qk)
+                if (warp_wait(&bars.a_done[pg], par, abortp)) {
+                    if (pt == 0) KDA_TR(TR_PREP_A, s);
+                    tc_fence_after();
+                    uint32_t d[32];
+                    tmem_ld32(tPl, d);
+                    tmem_wait_ld();
+                    __syncwarp();
+                    const int r = lane;
+                    if (pw == 0) {
+                        const float bl = bars.beta_s[pg][r];
+                        float *at = reinterpret_cast<float *>(scr + SC_AT);
+#pragma unroll
+                        for (int i = 0; i < kStep; ++i)
+                            at[i * (kScRow / 4) + r] = i < r ? bl * __uint_as_float(d[i]) : 0.f;
+                    } else {
+#pragma unroll
+                        for (int kg = 0; kg < 4; ++kg) {
+                            float x[8];
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) {
+                                const int i = 8 * kg + t;
+                                x[t] = i <= r ? __uint_as_float(d[i]) : 0.f;
+                            }
+                            uint4 w;
+                            w.x = pack_bf16(x[0], x[1]);
+                            w.y = pack_bf16(x[2], x[3]);
+                            w.z = pack_bf16(x[4], x[5]);
+                            w.w = pack_bf16(x[6], x[7]);
+                            *reinterpret_cast<uint4 *>(scr + SC_AQ + core32_off(r, 8 * kg)) = w;
+                        }
+                    }
+                } else {
+                    fail(bars);
+                    ok = false;
+                }
+                tc_fence_before();
+            }
+            group_sync(bar_id);                                             // scratch written
+
+            // ---------------- T by right-looking forward substitution (solver warp; lane = column)
+            if (pw == solve_w && !*abortp) {
+                const int c = lane;
+                const float bc = bars.beta_s[pg][c];
+                float *at = reinterpret_cast<float *>(scr + SC_AT);
+                float acc[kStep], t[kStep];
+#pragma unroll
+                for (int r = 0; r < kStep; ++r) acc[r] = 0.f;
+#pragma unroll
+                for (int i = 0; i < kStep; ++i) {
+                    t[i] = (i == c) ? bc : -acc[i];
+#pragma unroll
+                    for (int r4 = (i + 1) & ~3; r4 < kStep; r4 += 4) {
+                        const float4 a = *reinterpret_cast<const float4 *>(at + i * (kScRow / 4) + r4);
+                        if (r4 > i) acc[r4] = fmaf(a.x, t[i], acc[r4]);
+                        if (r4 + 1 > i) acc[r4 + 1] = fmaf(a.y, t[i], acc[r4 + 1]);
+                        if (r4 + 2 > i) acc[r4 + 2] = fmaf(a.z, t[i], acc[r4 + 2]);
+                        if (r4 + 3 > i) acc[r4 + 3] = fmaf(a.w, t[i], acc[r4 + 3]);
+                    }
+                }
+                // T bf16: B operand of the Z and P products
+#pragma unroll
+                for (int kg = 0; kg < 4; ++kg) {
+                    uint4 w;
+                    w.x = pack_bf16(t[8 * kg], t[8 * kg + 1]);
+                    w.y = pack_bf16(t[8 * kg + 2], t[8 * kg + 3]);
+                    w.z = pack_bf16(t[8 * kg + 4], t[8 * kg + 5]);
+                    w.w = pack_bf16(t[8 * kg + 6], t[8 * kg + 7]);
+                    *reinterpret_cast<uint4 *>(scr + SC_TB + core32_off(c, 8 * kg)) = w;
+                }
+                fence_proxy_async_smem();
+            }
+            group_sync(bar_id);                                             // T written
+
+            // ---------------- Z = Kh^T T (cols 0-31) and P = causal(A_qk) T (cols 32-63)
+            if (iss && !*abortp) {
+                KDA_TR(TR_PREP_T, s);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk)
+                    mma_ss(tP, sdesc(slot_u + SL_G0 + 2048 * kk, SL_G1 - SL_G0, 1024, kLayoutSW128),
+                           sdesc(scr_u + SC_TB + 256 * kk, 128, 512, kLayoutNone), idZ, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk)
+                    mma_ss(tP + 32, sdesc(scr_u + SC_AQ + 256 * kk, 128, 512, kLayoutNone),
+                           sdesc(scr_u + SC_TB + 256 * kk, 128, 512, kLayoutNone), idA, kk > 0);
+                tc_commit(&bars.z_done[pg]);
+            }
+            // ---------------- [P ; Diag(delta) Z]: operand B of MMA2
+            if (warp_wait(&bars.z_done[pg], par, abortp)) {
+                if (pt == 0) KDA_TR(TR_PREP_Z, s);
+                tc_fence_after();
+                uint32_t zv[32];
+                tmem_ld32(tPl, zv);
+                tmem_wait_ld();
+                const int i = 32 * pw + lane;           // key channel
+                const float di = dlt[i];
+#pragma unroll
+                for (int kg = 0; kg < 4; ++kg) {
+                    uint4 w;
+                    w.x = pack_bf16(di * __uint_as_float(zv[8 * kg]), di * __uint_as_float(zv[8 * kg + 1]));
+                    w.y = pack_bf16(di * __uint_as_float(zv[8 * kg + 2]), di * __uint_as_float(zv[8 * kg + 3]));
+                    w.z = pack_bf16(di * __uint_as_float(zv[8 * kg + 4]), di * __uint_as_float(zv[8 * kg + 5]));
+                    w.w = pack_bf16(di * __uint_as_float(zv[8 * kg + 6]), di * __uint_as_float(zv[8 * kg + 7]));
+                    *reinterpret_cast<uint4 *>(slot + SL_B2 + core32_off(32 + i, 8 * kg)) = w;
+                }
+                if (pw == 0) {                          // lanes 0-31 hold the rows of P
+                    uint32_t pv[32];
+                    tmem_ld32(tPl + 32, pv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int kg = 0; kg < 4; ++kg) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(pv[8 * kg]), __uint_as_float(pv[8 * kg + 1]));
+                        w.y = pack_bf16(__uint_as_float(pv[8 * kg + 2]), __uint_as_float(pv[8 * kg + 3]));
+                        w.z = pack_bf16(__uint_as_float(pv[8 * kg + 4]), __uint_as_float(pv[8 * kg + 5]));
+                        w.w = pack_bf16(__uint_as_float(pv[8 * kg + 6]), __uint_as_float(pv[8 * kg + 7]));
+                        *reinterpret_cast<uint4 *>(slot + SL_B2 + core32_off(lane, 8 * kg)) = w;
+                    }
+                }
+            } else {
+                fail(bars);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (pt == 0) bars.stop[pg] = *abortp;
+            group_sync(bar_id);                                             // [P ; Z] written
+            if (pt == 0 && bars.stop[pg] == 0) {
+                mbar_arrive(&bars.b_ready[pg]);
+                KDA_TR(TR_PREP_B, s);
+            }
+            if (bars.stop[pg]) break;
+        }
+        if (iss && issued) {
+            tc_commit(&bars.drain_prep[pg]);
+            mbar_wait_drain(&bars.drain_prep[pg], 0, kWaitLimit);
+        }
+
     }
 
     tc_fence_before();

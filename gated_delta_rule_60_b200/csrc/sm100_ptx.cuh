@@ -96,10 +96,15 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parit
 }
 
 // How a bounded wait polls: 0 = try_wait (the hardware may suspend the
-// thread between polls), 1 = test_wait spin, 2 = try_wait with a short
-// suspend-time hint, 3 = test_wait with a short sleep between polls.
+// thread between polls for a system-dependent time), 1 = test_wait spin,
+// 2 = try_wait with an explicit suspend-time hint (the waiting thread sleeps
+// until the phase completes or the hint runs out, so it issues almost no
+// instructions while it waits), 3 = test_wait with a short sleep between polls.
 #ifndef KDA_MBAR_WAIT
-#define KDA_MBAR_WAIT 0
+#define KDA_MBAR_WAIT 2
+#endif
+#ifndef KDA_MBAR_HINT_NS
+#define KDA_MBAR_HINT_NS 10000
 #endif
 
 __device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity) {
@@ -110,7 +115,7 @@ __device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity) {
     __nanosleep(32);
     return false;
 #elif KDA_MBAR_WAIT == 2
-    return mbar_try_wait_hint(bar, parity, 64);
+    return mbar_try_wait_hint(bar, parity, KDA_MBAR_HINT_NS);
 #else
     return mbar_try_wait(bar, parity);
 #endif
@@ -133,6 +138,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
+// Bounded wait that ignores the abort flag: used when a CTA drains its own
+// copies and MMAs before it exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
+                                                unsigned long long limit_cycles) {
+    if (mbar_poll(bar, parity)) return true;
+    const unsigned long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_poll(bar, parity)) return true;
+        if ((it & 63u) == 0u && clock64() - t0 > limit_cycles) return false;
+    }
+}
+
 // ---------------------------------------------------------------- proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -146,6 +163,15 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map,
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y),
         "r"(z)
+        : "memory");
+}
+
+// L2 prefetch of one tile box (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 
