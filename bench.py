@@ -76,7 +76,7 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples every 200 ms while running."""
+    """nvidia-smi clock/throttle samples every 100 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
               "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -95,7 +95,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -270,16 +270,29 @@ def run_gpu(args):
     assert binding.kda_stream_status(stream) == binding.KDA_OK
 
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    _barrier(world)
-    torch.cuda.synchronize()
+
+    def keep_busy(seconds):
+        # untimed steps of the same work, so that the clock samples (every
+        # 100 ms) bracket a timed region that may be only tens of ms long
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            while time.perf_counter() - t0 < seconds:
+                for _ in range(4):
+                    step()
+                stream.synchronize()
+
     with ClockSampler(local) as clk:
+        keep_busy(0.6)
+        _barrier(world)
+        torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             ev[0].record(stream)
             for i in range(args.steps):
                 step()
                 ev[i + 1].record(stream)
         stream.synchronize()
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        keep_busy(0.3)
     _barrier(world)
     per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])

@@ -24,18 +24,21 @@
 // With Ke = Kr Diag(eps) = K e^b and Qe = Q e^b the step is exactly
 //   W = V - Ke S0,   S_next = Diag(gamma) S0 + Z W,   O = Qe S0 + P W.
 // On the tensor cores everything is transposed so that the 128 value
-// channels are the MMA M dimension (tensor-memory lanes), and S0 enters as
-// bf16(eps * S0)^T:
-//   MMA1  [(Ke S0)^T | (Qe S0)^T] = (eps S0)^T [Kr ; Qr]^T      (N = 64, K = 128)
+// channels are the MMA M dimension (tensor-memory lanes):
+//   MMA1  [(Ke S0)^T | (Qe S0)^T] = bf16(S0)^T [Ke ; Qe]^T       (N = 64, K = 128)
 //   MMA2  [O^T | S_next^T] += [V^T | -(Ke S0)^T] [P ; Z]^T      (N = 160, K = 2 x 32)
-// The fp32 state lives in tensor memory as the accumulator of MMA2: before
-// each step the scan warpgroup replaces it by gamma * S0^T (fp32, exact
-// decay) and writes the bf16 operand of MMA1.  Everything that does not
-// involve S0 (gate, decays, A_kk, A_qk, T, P, Z) is prepared ahead of time.
+// (Ke and Qe are Kr and Qr rescaled in place by eps once the A_kk / A_qk
+// product has read them.)  The fp32 state lives in tensor memory as the
+// accumulator of MMA2: before each step the scan warpgroup replaces it by
+// gamma * S0^T (fp32, exact decay) and writes the bf16 operand of MMA1.
+// Everything that does not involve S0 (gate, decays, A_kk, A_qk, T, P, Z,
+// Ke, Qe) is prepared ahead of time.
 //
 // CTA = one (sequence, head) chain, 512 threads:
 //   warps 0-3   scan warpgroup: one thread per value channel; thread 0
-//               issues the step products and the tile loads of every step.
+//               issues the step products, lane 0 of warp 1 the tile loads,
+//               lane 0 of warp 2 the L2 prefetches and the TMA stores of o
+//               (full steps go through a shared-memory staging tile).
 //   warps 4-15  three prep warpgroups, taking steps in turn: gate and decay,
 //               scaled operands (in place in the step's tile slot), the
 //               A_kk / A_qk product, forward substitution for T, P, the Z
@@ -75,19 +78,24 @@ constexpr uint32_t SL_G0 = 16384, SL_G1 = 20480, SL_V0 = 24576, SL_V1 = 28672;
 constexpr uint32_t SL_B2 = 32768;
 constexpr uint32_t kSlotBytes = 43008;
 // Solve scratch of a prep warpgroup.
+// The P product reads 128 rows of its A operand causal(A_qk) (only the first
+// 32 are used); the other rows fall on the rest of this scratch region.
 constexpr uint32_t kScRow = 144;      // bytes per row of the fp32 scratch matrix (36 floats)
-constexpr uint32_t SC_AT = 0;         // (Diag(beta) strict_lower(A_kk))^T, fp32 [32][36]
-constexpr uint32_t SC_TB = 4608;      // T bf16, K-major no swizzle (row = column of T): B of Z and P
-constexpr uint32_t SC_AQ = 6656;      // causal(A_qk) bf16, K-major no swizzle: A of the P product
+constexpr uint32_t SC_AQ = 0;         // causal(A_qk) bf16, K-major no swizzle: A of the P product
+constexpr uint32_t SC_AT = 2048;      // (Diag(beta) strict_lower(A_kk))^T, fp32 [32][36]
+constexpr uint32_t SC_TB = 6656;      // T bf16, K-major no swizzle (row = column of T): B of Z and P
 constexpr uint32_t kScBytes = 8704;
+static_assert(SC_AQ + 128 * 64 <= kScBytes, "P product operand rows");
 constexpr uint32_t SM_SLOT = 0;
 constexpr uint32_t SM_SC = SM_SLOT + kSlots * kSlotBytes;
 constexpr uint32_t SM_GAMMA = SM_SC + kPrep * kScBytes;      // kSlots x 128 fp32
 constexpr uint32_t SM_EPS = SM_GAMMA + kSlots * 512;         // kSlots x 128 fp32
 constexpr uint32_t SM_DELTA = SM_EPS + kSlots * 512;         // kPrep x 128 fp32
-// The P product reads 128 rows of its A operand (only the first 32 are
-// causal(A_qk)); the tail pad keeps the other rows inside the allocation.
-constexpr uint32_t kSmemBytes = SM_DELTA + kPrep * 512 + 8192;
+// Output staging for the TMA stores of o: 2 steps x [32 tokens][64 ch] x 2,
+// 128B swizzle.
+constexpr uint32_t SM_OST = (SM_DELTA + kPrep * 512 + 1023) / 1024 * 1024;
+constexpr uint32_t kOstBytes = 8192;
+constexpr uint32_t kSmemBytes = SM_OST + 2 * kOstBytes;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSlotBytes % 1024 == 0, "slot alignment");
 
@@ -95,7 +103,7 @@ static_assert(kSlotBytes % 1024 == 0, "slot alignment");
 constexpr uint32_t COL_UP = 0;       // 32: (Ke S0)^T
 constexpr uint32_t COL_O = 32;       // 32: O^T
 constexpr uint32_t COL_S = 64;       // 128: S^T accumulator
-constexpr uint32_t COL_S16 = 192;    // 64: bf16 (eps S)^T, A operand of MMA1
+constexpr uint32_t COL_S16 = 192;    // 64: bf16 S^T, A operand of MMA1
 constexpr uint32_t COL_UN = 256;     // 16: bf16 -(Ke S0)^T, A operand of MMA2
 constexpr uint32_t COL_PREP = 288;   // kPrep x 64: prep accumulators (A_kk | A_qk, then Z | P)
 constexpr uint32_t kTmemCols = 512;
@@ -108,7 +116,8 @@ constexpr unsigned long long kWaitLimit = 1ull << 32;
 // Stage timestamps (clock64) of the chain run by CTA 0; a profiling build only.
 enum { TR_SCAN_ISSUE = 0, TR_SCAN_U, TR_SCAN_DONE, TR_SCAN_READY, TR_PREP_FULL, TR_PREP_P1,
        TR_PREP_A, TR_PREP_T, TR_PREP_Z, TR_PREP_B,
-       TR_S_M1, TR_S_UST, TR_S_BR, TR_S_LD, TR_S_H0, TR_S_H1, TR_S_OLD, TR_EVENTS };
+       TR_S_M1, TR_S_UST, TR_S_BR, TR_S_LD, TR_S_H0, TR_S_H1, TR_S_OLD, TR_S_FENCE, TR_S_ISSUED,
+       TR_EVENTS };
 constexpr int kTraceLen = 256;
 __device__ unsigned long long g_trace[TR_EVENTS][kTraceLen];
 __device__ unsigned long long g_cta_time[1024][3];   // globaltimer start, end, smid
@@ -321,6 +330,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v,
                        const __grid_constant__ CUtensorMap map_g,
+                       const __grid_constant__ CUtensorMap map_o,
                        const Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
@@ -423,10 +433,9 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             for (int s = kSlots; s < 2 * kSlots && s < nS; ++s) prefetch_step(s);
         bool alive = nS > 0;
         if (alive) {
-            // initial state: gamma_0 * S0 (fp32) and bf16(eps_0 * S0)
+            // initial state: gamma_0 * S0 (fp32) and bf16(S0)
             if (warp_wait(&bars.b_ready[0], 0, abortp)) {
                 const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA);
-                const float4 *e4 = reinterpret_cast<const float4 *>(sm + SM_EPS);
 #pragma unroll 1
                 for (int part = 0; part < 4; ++part) {
                     float s0[32];
@@ -439,9 +448,9 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                     uint32_t sb[16], y[32];
 #pragma unroll
                     for (int q4 = 0; q4 < 8; ++q4) {
-                        const float4 gm = g4[8 * part + q4], ep = e4[8 * part + q4];
-                        sb[2 * q4] = pack_bf16(ep.x * s0[4 * q4], ep.y * s0[4 * q4 + 1]);
-                        sb[2 * q4 + 1] = pack_bf16(ep.z * s0[4 * q4 + 2], ep.w * s0[4 * q4 + 3]);
+                        const float4 gm = g4[8 * part + q4];
+                        sb[2 * q4] = pack_bf16(s0[4 * q4], s0[4 * q4 + 1]);
+                        sb[2 * q4 + 1] = pack_bf16(s0[4 * q4 + 2], s0[4 * q4 + 3]);
                         y[4 * q4] = __float_as_uint(gm.x * s0[4 * q4]);
                         y[4 * q4 + 1] = __float_as_uint(gm.y * s0[4 * q4 + 1]);
                         y[4 * q4 + 2] = __float_as_uint(gm.z * s0[4 * q4 + 2]);
@@ -466,31 +475,66 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                                             : ((ch.h0_identity && row == j) ? 1.f : 0.f);
         }
 
-        uint32_t ov[32];                // outputs of the previous step, stored after the next MMA1 issue
-        int o_step = -1;
+        // Outputs of a step are held in registers until the next MMA1 has
+        // been issued.  A full step goes through shared memory and a TMA
+        // store (issued by lane 0 of warp 2 after the next barrier); the last,
+        // partial step of a sequence is written with masked plain stores.
+        uint32_t ov[32];
+        int o_step = -1, o_staged = -1, o_stored = -1;
+        const bool o_issuer = tid == 64;
         auto store_o = [&]() {
-            if (o_step < 0 || !ch.write_o) return;
+            if (o_step < 0 || !ch.write_o) { o_step = -1; return; }
             const int Lc = L - kStep * o_step;
-            __nv_bfloat16 *dst = p.o + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
-            const size_t step = (size_t)p.H * kD;
+            if (Lc >= kStep) {
+                // lanes j, j ^ 1 swap half of their tokens so that each writes
+                // 32-bit words (channels j & ~1, j | 1) of 16 tokens
+                unsigned char *st = sm + SM_OST + (o_step & 1) * kOstBytes + (j >> 6) * 4096;
+                const bool odd = j & 1;
+                const int r_base = odd ? 16 : 0;
 #pragma unroll
-            for (int r = 0; r < kStep; ++r)
-                if (r < Lc) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov[r]));
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t mine = odd ? ov[16 + i] : ov[i];    // token r_base + i, own channel
+                    const uint32_t give = odd ? ov[i] : ov[16 + i];    // the partner writes that token
+                    const uint32_t got = __shfl_xor_sync(0xffffffffu, give, 1);
+                    const float lo = __uint_as_float(odd ? got : mine), hi = __uint_as_float(odd ? mine : got);
+                    *reinterpret_cast<uint32_t *>(st + sw128_off(r_base + i, (j & 63) & ~1)) = pack_bf16(lo, hi);
+                }
+                fence_proxy_async_smem();
+                o_staged = o_step;
+            } else {
+                __nv_bfloat16 *dst = p.o + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
+                const size_t step = (size_t)p.H * kD;
+#pragma unroll
+                for (int r = 0; r < kStep; ++r)
+                    if (r < Lc) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov[r]));
+            }
             o_step = -1;
+        };
+        // after a barrier that follows store_o: write the staged step to global memory
+        auto flush_o = [&]() {
+            if (!o_issuer || o_staged <= o_stored) return;
+            const unsigned char *st = sm + SM_OST + (o_staged & 1) * kOstBytes;
+            const int z = (int)(start + (int64_t)kStep * o_staged);
+            tma_store_3d(&map_o, st, 0, h, z);
+            tma_store_3d(&map_o, st + 4096, 64, h, z);
+            bulk_commit_group();
+            o_stored = o_staged;
         };
         for (int c = 0; alive && c < nS; ++c) {
             const int sl = c % kSlots;
             const uint32_t slot_u = s_base + SM_SLOT + sl * kSlotBytes;
-            // ---- MMA1: [(Ke S)^T | (Qe S)^T] = bf16(eps S)^T [Kr ; Qr]^T, then the v part of MMA2
+            // ---- MMA1: [(Ke S)^T | (Qe S)^T] = bf16(S)^T [Ke ; Qe]^T, then the v part of MMA2
             if (tid == 0 && !*abortp) {
                 KDA_TR(TR_SCAN_ISSUE, c);
                 tc_fence_after();
+                KDA_TR(TR_S_FENCE, c);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tm + COL_UP, tm + COL_S16 + 8 * kk,
                            sdesc(slot_u + (kk >> 2) * SL_K1 + (kk & 3) * 32, 16, 1024, kLayoutSW128),
                            id1, kk > 0);
                 tc_commit(&bars.mma1_done);
+                KDA_TR(TR_S_ISSUED, c);
                 if (!ch.v_zero) {
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
@@ -503,7 +547,6 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             // request step c - 1 + kSlots (overlaps the MMA1 round trip)
             if (loader && c >= 1 && c - 1 + kSlots < nS && !*abortp) load_step(c - 1 + kSlots);
             if (prefetcher && c >= 1 && c - 1 + 2 * kSlots < nS) prefetch_step(c - 1 + 2 * kSlots);
-            store_o();
             // ---- -(Ke S)^T in bf16: A operand of the second half of MMA2
             if (warp_wait(&bars.mma1_done, c & 1, abortp)) {
                 if (tid == 0) KDA_TR(TR_S_M1, c);
@@ -520,8 +563,12 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             } else {
                 fail(bars);
             }
+            // staged outputs flushed before this barrier have left shared memory,
+            // so the buffer the next store_o writes is free
+            if (o_issuer) bulk_wait_group_read<0>();
             tc_fence_before();
             group_sync(1);
+            if (!*abortp) flush_o();
             if (tid == 0 && !*abortp) {
                 KDA_TR(TR_SCAN_U, c);
                 tc_fence_after();
@@ -531,6 +578,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                            sdesc(slot_u + SL_B2 + 256 * kk, 128, 512, kLayoutNone), id2, 1);
                 tc_commit(&bars.d_done);
             }
+            store_o();                      // outputs of step c - 1, during the MMA2 round trip
             // ---- step done: outputs, next step's operands (or the final state)
             if (warp_wait(&bars.d_done, c & 1, abortp)) {
                 tc_fence_after();
@@ -542,7 +590,6 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (tid == 0) KDA_TR(TR_S_BR, c);
                 const int sn = (c + 1) % kSlots;
                 const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA + sn * 512);
-                const float4 *e4 = reinterpret_cast<const float4 *>(sm + SM_EPS + sn * 512);
 #pragma unroll 1
                 for (int qt = 0; qt < 4 && ready; ++qt) {       // 32 key channels at a time
                     uint32_t sv[32];
@@ -553,14 +600,12 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                         uint32_t sb[16];
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 gm = g4[8 * qt + q4], ep = e4[8 * qt + q4];
+                            const float4 gm = g4[8 * qt + q4];
                             uint32_t *y = sv + 4 * q4;
                             const float2 s01 = make_float2(__uint_as_float(y[0]), __uint_as_float(y[1]));
                             const float2 s23 = make_float2(__uint_as_float(y[2]), __uint_as_float(y[3]));
-                            const float2 e01 = fmul2(make_float2(ep.x, ep.y), s01);
-                            const float2 e23 = fmul2(make_float2(ep.z, ep.w), s23);
-                            sb[2 * q4] = pack_bf16(e01.x, e01.y);
-                            sb[2 * q4 + 1] = pack_bf16(e23.x, e23.y);
+                            sb[2 * q4] = pack_bf16(s01.x, s01.y);
+                            sb[2 * q4 + 1] = pack_bf16(s23.x, s23.y);
                             const float2 g01 = fmul2(make_float2(gm.x, gm.y), s01);
                             const float2 g23 = fmul2(make_float2(gm.z, gm.w), s23);
                             y[0] = __float_as_uint(g01.x);
@@ -595,7 +640,14 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             alive = bars.stop[kPrep] == 0;
         }
-        store_o();                          // outputs of the last step
+        // outputs still pending: the staged step and the last step
+        if (o_issuer) bulk_wait_group_read<0>();
+        group_sync(1);
+        if (!*abortp) flush_o();
+        store_o();
+        group_sync(1);
+        if (!*abortp) flush_o();
+        if (o_issuer) bulk_wait_group<0>();
         if (tid == 0 && issued) {
             tc_commit(&bars.drain_scan);
             mbar_wait_drain(&bars.drain_scan, 0, kWaitLimit);
@@ -625,6 +677,14 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         constexpr uint32_t idA = idesc_bf16(128, 32, false, false);
         constexpr uint32_t idZ = idesc_bf16(128, 32, true, false);
 
+        // beta of this warpgroup's next step, loaded one step ahead (warp 0)
+        auto load_beta = [&](int s) {
+            const int Ls = min(kStep, L - kStep * s);
+            const int64_t tok = start + (int64_t)kStep * s + lane;
+            return lane < Ls ? __bfloat162float(p.beta[(size_t)tok * p.H + h]) : 0.f;
+        };
+        float beta_pre = (pw == 0 && pg < nS) ? load_beta(pg) : 0.f;
+
         for (int s = pg, u = 0; s < nS; s += kPrep, ++u) {
             const int sl = s % kSlots;
             unsigned char *slot = sm + SM_SLOT + sl * kSlotBytes;
@@ -632,9 +692,8 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             const int Ls = min(kStep, L - kStep * s);
             const uint32_t par = u & 1;
             if (pw == 0) {
-                const int64_t tok = start + (int64_t)kStep * s + lane;
-                bars.beta_s[pg][lane] =
-                    lane < Ls ? __bfloat162float(p.beta[(size_t)tok * p.H + h]) : 0.f;
+                bars.beta_s[pg][lane] = beta_pre;
+                if (s + kPrep < nS) beta_pre = load_beta(s + kPrep);
             }
             bool ok = warp_wait(&bars.slot_full[sl], (s / kSlots) & 1, abortp);
             if (!ok) fail(bars);
@@ -759,6 +818,21 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                     mma_ss(tP + 32, sdesc(scr_u + SC_AQ + 256 * kk, 128, 512, kLayoutNone),
                            sdesc(scr_u + SC_TB + 256 * kk, 128, 512, kLayoutNone), idA, kk > 0);
                 tc_commit(&bars.z_done[pg]);
+            }
+            // ---------------- Ke = Kr Diag(eps), Qe = Qr Diag(eps) in place (the A_kk /
+            // A_qk product has read Kr and Qr; the Z and P products do not use them)
+            if (!*abortp) {
+                const int kb = pw & 1, cc = 2 * lane, r0 = 16 * (pw >> 1);
+                const float2 ep = *reinterpret_cast<const float2 *>(sm + SM_EPS + sl * 512 + 4 * (64 * kb + cc));
+                unsigned char *tk = slot + (kb ? SL_K1 : SL_K0), *tq = slot + (kb ? SL_Q1 : SL_Q0);
+#pragma unroll
+                for (int rr = 0; rr < kTile; ++rr) {
+                    const uint32_t o = sw128_off(r0 + rr, cc);
+                    const float2 kv = fmul2(bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(tk + o)), ep);
+                    const float2 qv = fmul2(bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(tq + o)), ep);
+                    *reinterpret_cast<uint32_t *>(tk + o) = pack_bf16(kv.x, kv.y);
+                    *reinterpret_cast<uint32_t *>(tq + o) = pack_bf16(qv.x, qv.y);
+                }
             }
             // ---------------- [P ; Diag(delta) Z]: operand B of MMA2
             if (warp_wait(&bars.z_done[pg], par, abortp)) {
@@ -950,10 +1024,11 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
                                   const void *beta, const float *h0, const int32_t *cu, int N,
                                   int64_t T_tot, int H, void *o, float *hT, void *workspace,
                                   cudaStream_t s) {
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv, mg, mo;
     const int64_t T_map = T_tot > 0 ? T_tot : 1;
     if (!make_qkvg_map(&mq, q, H, T_map) || !make_qkvg_map(&mk, k, H, T_map) ||
-        !make_qkvg_map(&mv, v, H, T_map) || !make_qkvg_map(&mg, g, H, T_map))
+        !make_qkvg_map(&mv, v, H, T_map) || !make_qkvg_map(&mg, g, H, T_map) ||
+        !make_qkvg_map(&mo, o, H, T_map))
         return KDA_ERR_CUDA;
     auto kern = prefill::chunk_fwd_sm100_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -974,7 +1049,7 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.ws_R = p.ws_M = p.ws_S = nullptr;
     const SegPlan pl = plan_segments(N, T_tot, H);
     if (pl.G <= 1) {
-        kern<<<(unsigned)(N * H), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, p);
+        kern<<<(unsigned)(N * H), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);
         return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
     // one long sequence per head: local pass, combine, final pass
@@ -986,7 +1061,7 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.ws_M = ws + per;
     p.ws_S = ws + 2 * per;
     p.mode = prefill::kModeSegLocal;
-    kern<<<(unsigned)(H * (2 * pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, p);
+    kern<<<(unsigned)(H * (2 * pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     const int comb_smem = 2 * prefill::kD * prefill::kD * (int)sizeof(float);
     if (cudaFuncSetAttribute(prefill::seg_combine_kernel,
@@ -995,7 +1070,7 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     prefill::seg_combine_kernel<<<(unsigned)H, 256, comb_smem, s>>>(p.ws_M, p.ws_R, p.ws_S, H, pl.G);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     p.mode = prefill::kModeSegFinal;
-    kern<<<(unsigned)(H * (pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, p);
+    kern<<<(unsigned)(H * (pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
