@@ -66,6 +66,17 @@ def test_bf16_d128_varlen_full_oracle():
     check(inp, o, hT)
 
 
+def test_bf16_d128_step_boundaries():
+    """Sequence lengths around the 32-token state steps, packed next to each
+    other: full steps leave through the staged tile stores, partial last steps
+    through masked stores that must not touch the next sequence's rows."""
+    lengths = [31, 32, 33, 63, 64, 65, 96, 1]
+    inp = inputs.make_prefill(lengths, 2, 128, 128, torch.bfloat16, seed=42,
+                              h0_std=0.02)
+    o, hT = run(inp)
+    check(inp, o, hT)
+
+
 def test_bf16_d128_no_h0_no_hT():
     inp = inputs.make_prefill([48, 31], 2, 128, 128, torch.bfloat16, seed=41)
     o, hT = run(inp, output_final_state=False)
