@@ -18,6 +18,10 @@ inline bool aligned16(const void *p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
+// Largest T_tot of the bf16 d = 128 path: the last 32-token box must start
+// below 2^31.
+constexpr int64_t kMaxTokensSm100 = 0x7fffffc0;
+
 inline bool supported_simt_d(int d) {
     return d == 16 || d == 32 || d == 64 || d == 128;
 }
@@ -87,7 +91,7 @@ const char *kda_status_string(kda_status s) {
     switch (s) {
     case KDA_OK: return "ok";
     case KDA_ERR_INVALID_ARGUMENT: return "invalid argument";
-    case KDA_ERR_UNSUPPORTED: return "unsupported dtype or head size";
+    case KDA_ERR_UNSUPPORTED: return "unsupported dtype, head size or length";
     case KDA_ERR_WORKSPACE: return "workspace missing or too small";
     case KDA_ERR_CUDA: return "CUDA runtime error";
     case KDA_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
@@ -113,6 +117,8 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
     if (N < 0 || T_tot < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
     if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
     if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
+    // The tensor-core path addresses tokens with signed 32-bit TMA coordinates.
+    if (dt == KDA_BF16 && dk == 128 && T_tot > kMaxTokensSm100) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return T_tot == 0 ? KDA_OK : KDA_ERR_INVALID_ARGUMENT;
     if (cu_seqlens == nullptr && (T_tot % N) != 0) return KDA_ERR_INVALID_ARGUMENT;
     if ((int64_t)N * H > 0x7fffffff) return KDA_ERR_INVALID_ARGUMENT;

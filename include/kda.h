@@ -40,7 +40,9 @@
  *   - Support: KDA_BF16 with dk = dv = 128 runs the tcgen05 tensor-core
  *     path; KDA_BF16 with dk = dv in {16, 32, 64} and KDA_FP32 with
  *     dk = dv in {16, 32, 64, 128} run an fp32 CUDA-core path (the fp32 test
- *     mode).  Anything else returns KDA_ERR_UNSUPPORTED.
+ *     mode).  Anything else returns KDA_ERR_UNSUPPORTED, and so does a
+ *     tensor-core call with T_tot > 2^31 - 64 (tokens are signed 32-bit
+ *     TMA coordinates there).
  */
 #ifndef KDA_H
 #define KDA_H

@@ -88,16 +88,23 @@ def test_chunk_fwd_host_validation(lib):
     assert _call_fwd(lib, dt=7) == E.KDA_ERR_UNSUPPORTED
     assert _call_fwd(lib, N=0, T=0) == E.KDA_OK                    # nothing to do
     assert _call_fwd(lib, N=0, T=4) == E.KDA_ERR_INVALID_ARGUMENT
+    # the tensor-core path takes tokens as signed 32-bit TMA coordinates
+    assert _call_fwd(lib, T=1 << 31, dk=128, dv=128, dt=0) == E.KDA_ERR_UNSUPPORTED
 
 
 def test_chunk_fwd_workspace_validation(lib):
-    need = lib.kda_chunk_fwd_workspace_size(1, 8192, 96, 128, 128, 0)
-    if need == 0:
-        pytest.skip("this configuration needs no workspace")
-    st = _call_fwd(lib, T=8192, H=96, dk=128, dv=128, dt=0, ws=None, wsb=0)
+    # one 1M-token sequence on 8 heads is split into segments, which need scratch
+    T, H = 1 << 20, 8
+    need = lib.kda_chunk_fwd_workspace_size(1, T, H, 128, 128, 0)
+    assert need > 0
+    st = _call_fwd(lib, T=T, H=H, dk=128, dv=128, dt=0, ws=None, wsb=0)
     assert st == binding.KDA_ERR_WORKSPACE
-    st = _call_fwd(lib, T=8192, H=96, dk=128, dv=128, dt=0, ws=256, wsb=need - 1)
+    st = _call_fwd(lib, T=T, H=H, dk=128, dv=128, dt=0, ws=256, wsb=need - 1)
     assert st == binding.KDA_ERR_WORKSPACE
+    st = _call_fwd(lib, T=T, H=H, dk=128, dv=128, dt=0, ws=128, wsb=need)   # not 256-aligned
+    assert st == binding.KDA_ERR_WORKSPACE
+    # many heads fill the GPU without splitting: no scratch
+    assert lib.kda_chunk_fwd_workspace_size(1, 8192, 96, 128, 128, 0) == 0
 
 
 def test_decode_host_validation(lib):
