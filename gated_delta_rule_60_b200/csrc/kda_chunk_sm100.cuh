@@ -227,6 +227,41 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
     return c;
 }
 
+// Chains of a packed batch start longest first: CTA b runs head b % H of the
+// sequence whose length ranks b / H in decreasing order (ties by index).
+// Blocks are dispatched in index order, so the long chains fill the first
+// waves and the tail is made of short ones (longest-processing-time list
+// scheduling).  The rank of every sequence is computed by each CTA from the
+// lengths in shared memory, which is cheap for the batch sizes below.
+constexpr int kOrderMaxSeqs = 512;
+static_assert(kOrderMaxSeqs <= kThreads, "one sequence per thread when ranking");
+
+__device__ __forceinline__ int longest_first_cta(const Params &p, int tid) {
+    __shared__ int len_s[kOrderMaxSeqs];
+    __shared__ int pick;
+    if (tid == 0) pick = 0;
+    if (tid < p.N) {
+        const int64_t d = (int64_t)p.cu[tid + 1] - p.cu[tid];
+        len_s[tid] = d < 0 ? -1 : (d > 0x7fffffff ? 0x7fffffff : (int)d);
+    }
+    __syncthreads();
+    // (length descending, index ascending) is a strict total order, so the
+    // ranks are a permutation of [0, N) whatever the lengths are, and
+    // exactly one thread finds the wanted rank.
+    const int want = (int)(blockIdx.x / p.H);
+    if (tid < p.N) {
+        const int li = len_s[tid];
+        int rank = 0;
+        for (int j = 0; j < p.N; ++j) {
+            const int lj = len_s[j];
+            rank += (lj > li) | ((lj == li) & (j < tid));
+        }
+        if (rank == want) pick = tid;
+    }
+    __syncthreads();
+    return pick * p.H + (int)(blockIdx.x % p.H);
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -349,7 +384,9 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         g_cta_time[blockIdx.x][2] = sid & 0xffffffffu;
     }
 #endif
-    const Chain ch = chain_of(p, blockIdx.x);
+    const bool reorder = p.mode == kModeChains && p.cu != nullptr && p.N > 1 &&
+                         p.N <= kOrderMaxSeqs;
+    const Chain ch = chain_of(p, reorder ? longest_first_cta(p, tid) : (int)blockIdx.x);
     const int h = ch.h;
     const int64_t start = ch.start;
     const int L = ch.L;

@@ -66,6 +66,19 @@ def test_bf16_d128_varlen_full_oracle():
     check(inp, o, hT)
 
 
+@pytest.mark.parametrize("n_seq", [40, 600])
+def test_bf16_d128_many_sequences(n_seq):
+    """Many short sequences in one call: chains run longest first up to 512
+    sequences and in index order beyond; both orders must give every
+    (sequence, head) its own result."""
+    gen = np.random.default_rng(44 + n_seq)
+    lengths = gen.integers(0, 41, size=n_seq).tolist()
+    inp = inputs.make_prefill(lengths, 1, 128, 128, torch.bfloat16, seed=44,
+                              h0_std=0.02)
+    o, hT = run(inp)
+    check(inp, o, hT)
+
+
 def test_bf16_d128_step_boundaries():
     """Sequence lengths around the 32-token state steps, packed next to each
     other: full steps leave through the staged tile stores, partial last steps
@@ -197,11 +210,12 @@ def test_decode_equals_prefill():
         assert rel_err(S, hT.cpu().double().numpy()) <= tol_s
 
 
-def test_bad_seqlens_reported_not_faulted():
-    inp = inputs.make_prefill([32, 32], 2, 16, 16, torch.float32, seed=95)
+@pytest.mark.parametrize("dtype,dim", [(torch.float32, 16), (torch.bfloat16, 128)])
+def test_bad_seqlens_reported_not_faulted(dtype, dim):
+    inp = inputs.make_prefill([32, 32], 2, dim, dim, dtype, seed=95)
     d = to_device(inp)
     bad = torch.tensor([0, 40, 30], dtype=torch.int32, device="cuda")
-    o = torch.zeros(64, 2, 16, device="cuda")
+    o = torch.zeros(64, 2, dim, dtype=dtype, device="cuda")
     binding.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, bad, o=o)
     assert binding.kda_stream_status() == binding.KDA_ERR_BAD_SEQLENS
     assert binding.kda_stream_status() == binding.KDA_OK  # cleared
