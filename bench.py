@@ -159,9 +159,20 @@ def _max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _config(T, H, d):
+    """The workload both arms report (the reference arm runs a head sample
+    of it and says so in its cpu_baseline)."""
+    return {"workload": "k3_prefill B=1 H=96 T=8192 d=128 bf16 S0=0, "
+                        "chunk 16, one kda_chunk_fwd per step",
+            "tokens_per_gpu": T, "heads": H, "head_dim": d,
+            "l2": "inputs ~1 GB > L2 (126 MB), no flush",
+            "parallelism": "replicas: independent heads/sequences per GPU"}
 
 
 def _oracle_sample(seconds_target=12.0):
@@ -218,8 +229,7 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "k3_prefill B=1 H=96 T=8192 d=128 bf16 S0=0 "
-                               "(oracle on a head sample)"},
+        "config": _config(w.T_tot, w.H, w.dk),
         "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
@@ -480,11 +490,7 @@ def _report(args, world, rank, value, ms_step, achieved, hbm_peak, peak_kind, al
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "k3_prefill B=1 H=96 T=8192 d=128 bf16 S0=0, "
-                               "chunk 16, one kda_chunk_fwd per step",
-                   "tokens_per_gpu": T, "heads": H, "head_dim": d,
-                   "l2": "inputs ~1 GB > L2 (126 MB), no flush",
-                   "parallelism": "replicas: independent heads/sequences per GPU"},
+        "config": _config(T, H, d),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak,
                      "unit": "GB/s", "frac": achieved / hbm_peak,
                      "traffic": _measured_traffic(), "peak_source": peak_kind,

@@ -1,0 +1,106 @@
+"""Host-side logic of bench.py that needs no GPU: the multi-rank timing
+reduction over a world-2 gloo group, the reference arm's rank handling and
+JSON line, and the parsing of clock samples."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        # every rank times something different; all must report the slowest
+        got = bench._max_over_ranks(1.5 + 2.0 * rank, world)
+        bench._barrier(world)
+        with open(os.path.join(out_dir, "rank%d.json" % rank), "w") as f:
+            json.dump({"max": got}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_world2_gloo(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    for r in range(world):
+        with open(tmp_path / ("rank%d.json" % r)) as f:
+            assert json.load(f)["max"] == 1.5 + 2.0 * (world - 1)
+
+
+def _run_bench(args, env_extra, timeout=600):
+    env = dict(os.environ)
+    env.update(env_extra)
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args],
+                          capture_output=True, text=True, env=env, timeout=timeout)
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                   {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
+
+
+def test_reference_arm_line():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "3"],
+                   {"RANK": "0", "LOCAL_RANK": "0", "WORLD_SIZE": "1"})
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "Mtok/s"
+    assert line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["config"] == bench._config(8192, 96, 128)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "Mtok/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_clock_summary_parsing(tmp_path):
+    rows = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1830, 1965, 985.3, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+        "0, [N/A], 1965, 10, 0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    path = tmp_path / "clk.csv"
+    path.write_text("\n".join(rows) + "\n")
+    cs = bench.ClockSampler(0)
+    cs.path = str(path)
+    s = cs.summary()
+    assert s["sm_mhz"] == 1830.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    assert not path.exists()        # the temporary file is removed
+
+
+def test_default_run_on_cpu_fails_loudly():
+    """Without a GPU the product arm must not fall back to anything."""
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    r = _run_bench(["--steps", "1", "--warmup", "3"], {"WORLD_SIZE": "1"}, timeout=300)
+    assert r.returncode != 0
+    assert not any(ln.startswith("{") for ln in r.stdout.splitlines())
