@@ -63,7 +63,7 @@ extern "C" {
 typedef enum {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size     */
-    KDA_ERR_UNSUPPORTED = 2,      /* dtype / head size not in the matrix   */
+    KDA_ERR_UNSUPPORTED = 2,      /* dtype, head size or length not supported */
     KDA_ERR_WORKSPACE = 3,        /* workspace missing or too small        */
     KDA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed  */
     KDA_ERR_TIMEOUT = 5,          /* a kernel's bounded wait ran out       */
@@ -123,6 +123,8 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
  *   o           device [B, H, dv]     (dt) output, read from the updated S
  *
  * A single pass over S: every state element is read once and written once.
+ * Returns KDA_OK once the work is enqueued on `stream` (B = 0 enqueues
+ * nothing); argument errors as for kda_chunk_fwd.
  */
 KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const void *g, const void *beta, float *S,
