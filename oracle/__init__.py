@@ -41,6 +41,11 @@ def _load():
             ctypes.c_int, ctypes.c_int, dp]
         lib.kda_oracle_log_alpha.restype = ctypes.c_double
         lib.kda_oracle_log_alpha.argtypes = [ctypes.c_double]
+        lib.kda_oracle_backward.restype = ctypes.c_int
+        lib.kda_oracle_backward.argtypes = [
+            dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+            ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, dp, dp, dp, dp, dp, dp, dp, dp]
         _lib = lib
     return _lib
 
@@ -100,6 +105,46 @@ def forward(q, k, v, g, beta, cu_seqlens, h0=None, unit_mask=None,
     if rc != 0:
         raise ValueError("kda_oracle_forward: malformed cu_seqlens or OOM")
     return o, hT
+
+
+def backward(q, k, v, g, beta, cu_seqlens, h0=None, d_o=None, d_hT=None):
+    """fp64 gradient of the prefill, by the chain rule through the token
+    recurrence in reverse.
+
+    For L = <d_o, o> + <d_hT, hT> (either term may be None = zero) returns a
+    dict of numpy arrays: dq, dk, dg [T_tot, H, dk], dv [T_tot, H, dv],
+    dbeta [T_tot, H] and dh0 [N, H, dk, dv] (the gradient with respect to the
+    initial state, zero or not).
+    """
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    cu = np.ascontiguousarray(np.asarray(
+        cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+        dtype=np.int64))
+    T_tot, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu.shape[0] - 1
+    assert k.shape == (T_tot, H, dk) and g.shape == (T_tot, H, dk)
+    assert v.shape == (T_tot, H, dv) and beta.shape == (T_tot, H)
+    h0a = None if h0 is None else _f64(h0)
+    doa = None if d_o is None else _f64(d_o)
+    dha = None if d_hT is None else _f64(d_hT)
+    if h0a is not None:
+        assert h0a.shape == (N, H, dk, dv)
+    if doa is not None:
+        assert doa.shape == (T_tot, H, dv)
+    if dha is not None:
+        assert dha.shape == (N, H, dk, dv)
+    out = {"dq": np.zeros((T_tot, H, dk)), "dk": np.zeros((T_tot, H, dk)),
+           "dv": np.zeros((T_tot, H, dv)), "dg": np.zeros((T_tot, H, dk)),
+           "dbeta": np.zeros((T_tot, H)), "dh0": np.zeros((N, H, dk, dv))}
+    rc = _load().kda_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0a),
+        _ptr(cu, ctypes.c_int64), N, T_tot, H, dk, dv, _ptr(doa), _ptr(dha),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+        _ptr(out["dbeta"]), _ptr(out["dh0"]))
+    if rc != 0:
+        raise ValueError("kda_oracle_backward: malformed cu_seqlens or OOM")
+    return out
 
 
 def decode(q, k, v, g, beta, S):

@@ -32,6 +32,9 @@
  * query scale; q and k are used as given (their normalisation belongs to the
  * input); sequences restart from h0 (or zero) at each cu_seqlens boundary.
  *
+ * kda_oracle_backward (at the end of the file) is the gradient of the same
+ * prefill by the chain rule, token by token in reverse.
+ *
  * Layouts (row-major, last index contiguous), all fp64:
  *   q, k, g  [T_tot, H, dk]      v, o  [T_tot, H, dv]      beta [T_tot, H]
  *   h0, hT   [N, H, dk, dv]      cu_seqlens int64 [N+1]
@@ -162,3 +165,194 @@ int kda_oracle_decode(const double *q, const double *k, const double *v,
 
 /* The gate on its own, so tests can pin it against closed forms. */
 double kda_oracle_log_alpha(double g) { return log_alpha(g); }
+
+/* ------------------------------------------------------------------------
+ * Backward pass: the gradient of the prefill by the chain rule, token by
+ * token in reverse (the pages name training as the use of the chunked form:
+ * "Kimi K3 发布核实与 Moonshot AI 主干架构演变", §3 "KDA 为什么不同于 MLA",
+ * item 3).  Given dL/do_t and dL/dhT it returns dL/dq, dk, dv, dg, dbeta,
+ * dh0 for L = <dO, O> + <dhT, hT>.
+ * ---------------------------------------------------------------------- */
+
+/* d(log a)/dg = -5 sigmoid(g) (1 - sigmoid(g)); 0 at g = +/-inf. */
+static double dlog_alpha(double g)
+{
+    double s, c;   /* s = sigmoid(g), c = 1 - s = sigmoid(-g) */
+    if (g >= 0.0) {
+        double e = exp(-g);
+        s = 1.0 / (1.0 + e);
+        c = e / (1.0 + e);
+    } else {
+        double e = exp(g);
+        s = e / (1.0 + e);
+        c = 1.0 / (1.0 + e);
+    }
+    return -5.0 * s * c;
+}
+
+/*
+ * Adjoint of one token step.  P is the state before the token (S_{t-1}).
+ * On entry dS holds dL/dS_t from the later tokens (and hT); on exit it holds
+ * dL/dS_{t-1}.  dout may be NULL (no gradient on o_t).  work has room for
+ * 2 dk dv + 4 dv + dk doubles.  Forward quantities are recomputed from P:
+ *   S' = Diag(a) P,  r = S'^T k,  u = beta (v - r),  S_t = S' + k u^T,
+ *   o = S_t^T q.
+ */
+static void kda_token_backward(const double *P, int dk, int dv,
+                               const double *q, const double *k,
+                               const double *v, const double *g, double beta,
+                               const double *dout, double *dS, double *dq,
+                               double *dk_, double *dv_, double *dg,
+                               double *dbeta, double *work)
+{
+    double *Sp = work;                       /* S'   [dk][dv] */
+    double *St = Sp + (size_t)dk * dv;       /* S_t  [dk][dv] */
+    double *r = St + (size_t)dk * dv;        /* dv */
+    double *u = r + dv, *du = u + dv, *dr = du + dv;
+    double *a = dr + dv;                     /* dk */
+
+    /* recompute the forward step */
+    for (int i = 0; i < dk; ++i) {
+        a[i] = exp(log_alpha(g[i]));
+        for (int j = 0; j < dv; ++j)
+            Sp[(size_t)i * dv + j] = a[i] * P[(size_t)i * dv + j];
+    }
+    for (int j = 0; j < dv; ++j) r[j] = 0.0;
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) r[j] += Sp[(size_t)i * dv + j] * k[i];
+    for (int j = 0; j < dv; ++j) u[j] = beta * (v[j] - r[j]);
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j)
+            St[(size_t)i * dv + j] = Sp[(size_t)i * dv + j] + k[i] * u[j];
+
+    /* o = S_t^T q:  dq = S_t do,  dS_t += q do^T */
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        if (dout)
+            for (int j = 0; j < dv; ++j) acc += St[(size_t)i * dv + j] * dout[j];
+        dq[i] = acc;
+    }
+    if (dout)
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += q[i] * dout[j];
+
+    /* S_t = S' + k u^T:  du = dS_t^T k,  dk = dS_t u,  dS' = dS_t (+ below) */
+    for (int j = 0; j < dv; ++j) du[j] = 0.0;
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dv; ++j) {
+            du[j] += dS[(size_t)i * dv + j] * k[i];
+            acc += dS[(size_t)i * dv + j] * u[j];
+        }
+        dk_[i] = acc;
+    }
+
+    /* u = beta (v - r) */
+    double db = 0.0;
+    for (int j = 0; j < dv; ++j) {
+        db += du[j] * (v[j] - r[j]);
+        dv_[j] = beta * du[j];
+        dr[j] = -beta * du[j];
+    }
+    *dbeta = db;
+
+    /* r = S'^T k:  dk += S' dr,  dS' += k dr^T */
+    for (int i = 0; i < dk; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dv; ++j) {
+            acc += Sp[(size_t)i * dv + j] * dr[j];
+            dS[(size_t)i * dv + j] += k[i] * dr[j];
+        }
+        dk_[i] += acc;
+    }
+
+    /* S' = Diag(a) P:  da_i = sum_j dS'_ij P_ij,  dg_i = da_i a_i dlog_alpha(g_i),
+     * dP = Diag(a) dS' */
+    for (int i = 0; i < dk; ++i) {
+        double da = 0.0;
+        for (int j = 0; j < dv; ++j) {
+            da += dS[(size_t)i * dv + j] * P[(size_t)i * dv + j];
+            dS[(size_t)i * dv + j] *= a[i];
+        }
+        dg[i] = da * a[i] * dlog_alpha(g[i]);
+    }
+}
+
+/*
+ * Backward of kda_oracle_forward.  dO [T_tot,H,dv] and dhT [N,H,dk,dv] may
+ * be NULL (zero).  Outputs (all required except dh0, which may be NULL):
+ * dq, dk, dg [T_tot,H,dk], dv [T_tot,H,dv], dbeta [T_tot,H], dh0 [N,H,dk,dv].
+ * The states before each token are recomputed by the forward step from
+ * checkpoints kept every kCkpt tokens, so memory per unit stays small; the
+ * arithmetic is the same forward step.  Returns 0, or -1 on a malformed
+ * cu_seqlens or allocation failure.
+ */
+int kda_oracle_backward(const double *q, const double *k, const double *v,
+                        const double *g, const double *beta, const double *h0,
+                        const int64_t *cu_seqlens, int N, int64_t T_tot,
+                        int H, int dk, int dv, const double *dO,
+                        const double *dhT, double *dq, double *dk_,
+                        double *dv_, double *dg, double *dbeta, double *dh0)
+{
+    enum { kCkpt = 64 };
+    if (cu_seqlens[0] != 0 || cu_seqlens[N] != T_tot) return -1;
+    for (int n = 0; n < N; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    int err = 0;
+    long units = (long)N * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long u = 0; u < units; ++u) {
+        int n = (int)(u / H), h = (int)(u % H);
+        const int64_t t0 = cu_seqlens[n], t1 = cu_seqlens[n + 1];
+        const int64_t L = t1 - t0;
+        const int64_t nseg = (L + kCkpt - 1) / kCkpt;
+        const size_t sz = (size_t)dk * dv;
+        double *S = (double *)malloc(sizeof(double) * (2 * sz + dv));
+        double *ckpt = (double *)malloc(sizeof(double) * sz * (size_t)(nseg > 0 ? nseg : 1));
+        double *buf = (double *)malloc(sizeof(double) * sz * kCkpt);
+        double *work = (double *)malloc(sizeof(double) * (2 * sz + 4 * (size_t)dv + dk));
+        if (!S || !ckpt || !buf || !work) {
+            free(S); free(ckpt); free(buf); free(work);
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        double *dS = S + sz, *r = dS + sz;
+        /* forward, keeping the state before every kCkpt-th token */
+        if (h0) memcpy(S, h0 + (size_t)u * sz, sizeof(double) * sz);
+        else memset(S, 0, sizeof(double) * sz);
+        for (int64_t t = t0; t < t1; ++t) {
+            if ((t - t0) % kCkpt == 0)
+                memcpy(ckpt + (size_t)((t - t0) / kCkpt) * sz, S, sizeof(double) * sz);
+            size_t th = (size_t)t * H + h;
+            kda_token(S, dk, dv, q + th * dk, k + th * dk, v + th * dv,
+                      g + th * dk, beta[th], NULL, r);
+        }
+        /* reverse sweep */
+        if (dhT) memcpy(dS, dhT + (size_t)u * sz, sizeof(double) * sz);
+        else memset(dS, 0, sizeof(double) * sz);
+        for (int64_t sg = nseg - 1; sg >= 0; --sg) {
+            const int64_t a0 = t0 + sg * kCkpt;
+            const int64_t a1 = a0 + kCkpt < t1 ? a0 + kCkpt : t1;
+            memcpy(S, ckpt + (size_t)sg * sz, sizeof(double) * sz);
+            for (int64_t t = a0; t < a1; ++t) {
+                memcpy(buf + (size_t)(t - a0) * sz, S, sizeof(double) * sz);
+                size_t th = (size_t)t * H + h;
+                kda_token(S, dk, dv, q + th * dk, k + th * dk, v + th * dv,
+                          g + th * dk, beta[th], NULL, r);
+            }
+            for (int64_t t = a1 - 1; t >= a0; --t) {
+                size_t th = (size_t)t * H + h;
+                kda_token_backward(buf + (size_t)(t - a0) * sz, dk, dv,
+                                   q + th * dk, k + th * dk, v + th * dv,
+                                   g + th * dk, beta[th],
+                                   dO ? dO + th * dv : NULL, dS,
+                                   dq + th * dk, dk_ + th * dk, dv_ + th * dv,
+                                   dg + th * dk, dbeta + th, work);
+            }
+        }
+        if (dh0) memcpy(dh0 + (size_t)u * sz, dS, sizeof(double) * sz);
+        free(S); free(ckpt); free(buf); free(work);
+    }
+    return err ? -1 : 0;
+}
