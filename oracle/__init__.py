@@ -35,6 +35,11 @@ def _load():
             dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
             ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.POINTER(ctypes.c_uint8), dp, dp]
+        lib.kda_oracle_forward_gate.restype = ctypes.c_int
+        lib.kda_oracle_forward_gate.argtypes = \
+            lib.kda_oracle_forward.argtypes + [ctypes.c_int]
+        lib.kda_oracle_log_alpha_softplus.restype = ctypes.c_double
+        lib.kda_oracle_log_alpha_softplus.argtypes = [ctypes.c_double]
         lib.kda_oracle_decode.restype = ctypes.c_int
         lib.kda_oracle_decode.argtypes = [
             dp, dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
@@ -70,15 +75,25 @@ def log_alpha(g: float) -> float:
     return _load().kda_oracle_log_alpha(float(g))
 
 
+GATES = {"sigmoid5": 0, "softplus": 1}
+
+
+def log_alpha_softplus(g: float) -> float:
+    """log a = -softplus(g), the unbounded gate K3 replaced, in fp64."""
+    return _load().kda_oracle_log_alpha_softplus(float(g))
+
+
 def forward(q, k, v, g, beta, cu_seqlens, h0=None, unit_mask=None,
-            want_o=True):
+            want_o=True, gate="sigmoid5"):
     """Token-by-token fp64 prefill.
 
     q, k, g: [T_tot, H, dk]; v: [T_tot, H, dv]; beta: [T_tot, H];
     cu_seqlens: [N+1] integers; h0: [N, H, dk, dv] or None (= zeros);
-    unit_mask: bool [N, H] or None (= every unit).  Returns (o, hT) as fp64
-    numpy arrays [T_tot, H, dv] and [N, H, dk, dv]; entries of units that the
-    mask skips are NaN.
+    unit_mask: bool [N, H] or None (= every unit).  gate: "sigmoid5" for K3's
+    log a = -5 sigmoid(g), "softplus" for Kimi Linear's unbounded
+    log a = -softplus(g) (the variant the pages contrast it with).  Returns
+    (o, hT) as fp64 numpy arrays [T_tot, H, dv] and [N, H, dk, dv]; entries of
+    units that the mask skips are NaN.
     """
     q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
     cu = np.ascontiguousarray(np.asarray(
@@ -98,10 +113,10 @@ def forward(q, k, v, g, beta, cu_seqlens, h0=None, unit_mask=None,
                                     .reshape(N * H))
     o = np.full((T_tot, H, dv), np.nan) if want_o else None
     hT = np.full((N, H, dk, dv), np.nan)
-    rc = _load().kda_oracle_forward(
+    rc = _load().kda_oracle_forward_gate(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0a),
         _ptr(cu, ctypes.c_int64), N, T_tot, H, dk, dv,
-        _ptr(mask, ctypes.c_uint8), _ptr(o), _ptr(hT))
+        _ptr(mask, ctypes.c_uint8), _ptr(o), _ptr(hT), GATES[gate])
     if rc != 0:
         raise ValueError("kda_oracle_forward: malformed cu_seqlens or OOM")
     return o, hT

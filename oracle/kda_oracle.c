@@ -57,15 +57,32 @@ static double log_alpha(double g)
     return -5.0 * s;
 }
 
+/* The unbounded gate that K3 replaced (same page, same bullet: Kimi
+ * Linear's negative-softplus log-decay): log a = -softplus(g) = -log(1 + e^g),
+ * written so that g = -inf gives 0 and g = +inf gives -inf (a = 0). */
+static double log_alpha_softplus(double g)
+{
+    if (g > 0.0) return -(g + log1p(exp(-g)));
+    return -log1p(exp(g));
+}
+
+enum { GATE_SIGMOID5 = 0, GATE_SOFTPLUS = 1 };
+
+static double log_alpha_mode(double g, int gate)
+{
+    return gate == GATE_SOFTPLUS ? log_alpha_softplus(g) : log_alpha(g);
+}
+
 /* One token of the recurrence on one head's state S [dk][dv] (in place).
- * o may be NULL.  r is scratch of length dv. */
-static void kda_token(double *S, int dk, int dv,
-                      const double *q, const double *k, const double *v,
-                      const double *g, double beta, double *o, double *r)
+ * o may be NULL.  r is scratch of length dv.  gate selects the log-decay. */
+static void kda_token_gate(double *S, int dk, int dv,
+                           const double *q, const double *k, const double *v,
+                           const double *g, double beta, double *o, double *r,
+                           int gate)
 {
     /* decay first */
     for (int i = 0; i < dk; ++i) {
-        double a = exp(log_alpha(g[i]));
+        double a = exp(log_alpha_mode(g[i], gate));
         double *row = S + (size_t)i * dv;
         for (int j = 0; j < dv; ++j) row[j] *= a;
     }
@@ -94,18 +111,29 @@ static void kda_token(double *S, int dk, int dv,
     }
 }
 
+/* The token step with the K3 gate, log a = -5 sigmoid(g). */
+static void kda_token(double *S, int dk, int dv,
+                      const double *q, const double *k, const double *v,
+                      const double *g, double beta, double *o, double *r)
+{
+    kda_token_gate(S, dk, dv, q, k, v, g, beta, o, r, GATE_SIGMOID5);
+}
+
 /*
  * Prefill: every token of every (sequence n, head h) unit whose mask byte is
  * nonzero (mask may be NULL = all units).  Units are independent; OpenMP runs
- * them in parallel, the tokens of a unit run in order.
- * Returns 0, or -1 on a malformed cu_seqlens or allocation failure.
+ * them in parallel, the tokens of a unit run in order.  gate: 0 = the K3
+ * gate -5 sigmoid(g), 1 = the unbounded -softplus(g).
+ * Returns 0, or -1 on a malformed cu_seqlens, an unknown gate or allocation
+ * failure.
  */
-int kda_oracle_forward(const double *q, const double *k, const double *v,
-                       const double *g, const double *beta, const double *h0,
-                       const int64_t *cu_seqlens, int N, int64_t T_tot,
-                       int H, int dk, int dv, const uint8_t *unit_mask,
-                       double *o, double *hT)
+int kda_oracle_forward_gate(const double *q, const double *k, const double *v,
+                            const double *g, const double *beta, const double *h0,
+                            const int64_t *cu_seqlens, int N, int64_t T_tot,
+                            int H, int dk, int dv, const uint8_t *unit_mask,
+                            double *o, double *hT, int gate)
 {
+    if (gate != GATE_SIGMOID5 && gate != GATE_SOFTPLUS) return -1;
     if (cu_seqlens[0] != 0 || cu_seqlens[N] != T_tot) return -1;
     for (int n = 0; n < N; ++n)
         if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
@@ -127,13 +155,24 @@ int kda_oracle_forward(const double *q, const double *k, const double *v,
         else memset(S, 0, sizeof(double) * sz);
         for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
             size_t th = (size_t)t * H + h;
-            kda_token(S, dk, dv, q + th * dk, k + th * dk, v + th * dv,
-                      g + th * dk, beta[th], o ? o + th * dv : NULL, r);
+            kda_token_gate(S, dk, dv, q + th * dk, k + th * dk, v + th * dv,
+                           g + th * dk, beta[th], o ? o + th * dv : NULL, r, gate);
         }
         if (hT) memcpy(hT + (size_t)u * sz, S, sizeof(double) * sz);
         free(S);
     }
     return err ? -1 : 0;
+}
+
+/* Prefill with the K3 gate. */
+int kda_oracle_forward(const double *q, const double *k, const double *v,
+                       const double *g, const double *beta, const double *h0,
+                       const int64_t *cu_seqlens, int N, int64_t T_tot,
+                       int H, int dk, int dv, const uint8_t *unit_mask,
+                       double *o, double *hT)
+{
+    return kda_oracle_forward_gate(q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H,
+                                   dk, dv, unit_mask, o, hT, GATE_SIGMOID5);
 }
 
 /*
@@ -163,8 +202,9 @@ int kda_oracle_decode(const double *q, const double *k, const double *v,
     return err ? -1 : 0;
 }
 
-/* The gate on its own, so tests can pin it against closed forms. */
+/* The gates on their own, so tests can pin them against closed forms. */
 double kda_oracle_log_alpha(double g) { return log_alpha(g); }
+double kda_oracle_log_alpha_softplus(double g) { return log_alpha_softplus(g); }
 
 /* ------------------------------------------------------------------------
  * Backward pass: the gradient of the prefill by the chain rule, token by

@@ -6,7 +6,9 @@ exp(b_r - b_i) directly (no reciprocal scaling), so it cannot share a mistake
 with either the oracle or the CUDA path.
 
 For one head and a chunk of rows r = 1..C with start state S0 (dk x dv):
-  l_r   = -5 * sigmoid(g_r)                      (log-decay per key channel)
+  l_r   = -5 * sigmoid(g_r)                      (log-decay per key channel;
+                                                  -softplus(g_r) for the
+                                                  unbounded gate variant)
   b_r   = l_1 + ... + l_r                        (inclusive prefix sum)
   A_ri  = beta_r * sum_c k_rc k_ic exp(b_rc - b_ic)      for i < r, else 0
   T     = (I + A)^-1 Diag(beta)
@@ -20,16 +22,21 @@ exp(b_r - b_i) when row r reads it.)
 import numpy as np
 
 
-def _log_decay(g):
+def _log_decay(g, gate="sigmoid5"):
     with np.errstate(over="ignore"):
+        if gate == "softplus":          # -log(1 + e^g), stable for large |g|
+            return -(np.maximum(g, 0.0) + np.log1p(np.exp(-np.abs(g))))
         return -5.0 / (1.0 + np.exp(-g))
 
 
-def chunk_step(q, k, v, g, beta, S0):
+def chunk_step(q, k, v, g, beta, S0, gate="sigmoid5"):
     """One chunk.  q,k,g [C,dk]; v [C,dv]; beta [C]; S0 [dk,dv]."""
     C = q.shape[0]
-    b = np.cumsum(_log_decay(g), axis=0)                     # [C, dk]
-    ratio = np.exp(b[:, None, :] - b[None, :, :])           # [r, i, c]
+    b = np.cumsum(_log_decay(g, gate), axis=0)               # [C, dk]
+    # decay ratios for i <= r only (the others would be growth factors that
+    # the causal masks drop; forming them could overflow for an unbounded gate)
+    lower = np.tril(np.ones((C, C), dtype=bool))[:, :, None]
+    ratio = np.exp(np.where(lower, b[:, None, :] - b[None, :, :], -np.inf))
     kk = np.einsum("rc,ic,ric->ri", k, k, ratio)
     qk = np.einsum("rc,ic,ric->ri", q, k, ratio)
     strict = np.tril(np.ones((C, C)), -1)
@@ -42,7 +49,7 @@ def chunk_step(q, k, v, g, beta, S0):
     return O, S
 
 
-def forward(q, k, v, g, beta, cu_seqlens, h0=None, chunk=16):
+def forward(q, k, v, g, beta, cu_seqlens, h0=None, chunk=16, gate="sigmoid5"):
     """Whole packed batch, chunk by chunk.  Same layouts as the oracle."""
     q, k, v, g, beta = (np.asarray(x, dtype=np.float64)
                         for x in (q, k, v, g, beta))
@@ -59,7 +66,7 @@ def forward(q, k, v, g, beta, cu_seqlens, h0=None, chunk=16):
             for s in range(cu[n], cu[n + 1], chunk):
                 e = min(s + chunk, cu[n + 1])
                 O, S = chunk_step(q[s:e, h], k[s:e, h], v[s:e, h],
-                                  g[s:e, h], beta[s:e, h], S)
+                                  g[s:e, h], beta[s:e, h], S, gate)
                 o[s:e, h] = O
             hT[n, h] = S
     return o, hT

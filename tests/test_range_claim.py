@@ -121,3 +121,18 @@ def test_lost_precision_centred_vs_absolute():
     assert lost(centred) <= 0.01 * 32 * d
     assert abs(lost(centred) - expect) <= 2
     assert lost(centred[:31]) == 0
+
+
+def test_unbounded_gate_breaks_the_tile_range():
+    """The gate K3 replaced, log a = -softplus(g), has no lower bound: from
+    g of about 5.6 upwards one 16-token tile decays past e^{-88.7}, so the
+    reciprocal factor e^{-b} of that tile no longer fits bf16, while the
+    bounded gate stays at e^{80} for any g."""
+    softplus = lambda x: np.log1p(np.exp(x))
+    g = np.array([0.0, 3.0, 5.6, 8.0, 30.0])
+    tile = 16 * softplus(g)                       # -b over one tile
+    assert np.all(tile[2:] > math.log(BF16_MAX)) and np.all(tile[:2] < 80.0)
+    assert not torch.isfinite(to_bf16(np.exp(tile[2:]))).any()
+    bounded = -16 * log_decay(np.array([0.0, 5.6, 30.0, np.inf]))
+    assert np.all(bounded <= 80.0)
+    assert torch.isfinite(to_bf16(np.exp(bounded))).all()
