@@ -156,6 +156,7 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
     if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
     if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
     if (B == 0) return KDA_OK;
+    if ((int64_t)B * H > 0x7fffffff) return KDA_ERR_INVALID_ARGUMENT;
     const void *req[] = {q, k, v, g, beta, S, o};
     for (const void *p : req)
         if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;

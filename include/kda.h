@@ -101,6 +101,7 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t T_tot, int32_t H,
  *   workspace   device scratch of kda_chunk_fwd_workspace_size() bytes
  *               (may be NULL when that is 0); 256-byte aligned.
  *
+ * N * H must be below 2^31.
  * Returns KDA_OK once the work is enqueued on `stream`.  Malformed
  * cu_seqlens contents are found on the device: the affected sequences are
  * skipped and kda_stream_status() returns KDA_ERR_BAD_SEQLENS.
@@ -123,8 +124,8 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
  *   o           device [B, H, dv]     (dt) output, read from the updated S
  *
  * A single pass over S: every state element is read once and written once.
- * Returns KDA_OK once the work is enqueued on `stream` (B = 0 enqueues
- * nothing); argument errors as for kda_chunk_fwd.
+ * B * H must be below 2^31.  Returns KDA_OK once the work is enqueued on
+ * `stream` (B = 0 enqueues nothing); argument errors as for kda_chunk_fwd.
  */
 KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const void *g, const void *beta, float *S,

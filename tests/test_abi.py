@@ -88,6 +88,7 @@ def test_chunk_fwd_host_validation(lib):
     assert _call_fwd(lib, dt=7) == E.KDA_ERR_UNSUPPORTED
     assert _call_fwd(lib, N=0, T=0) == E.KDA_OK                    # nothing to do
     assert _call_fwd(lib, N=0, T=4) == E.KDA_ERR_INVALID_ARGUMENT
+    assert _call_fwd(lib, N=1 << 16, H=1 << 15, T=1 << 16) == E.KDA_ERR_INVALID_ARGUMENT
     # the tensor-core path takes tokens as signed 32-bit TMA coordinates
     assert _call_fwd(lib, T=1 << 31, dk=128, dv=128, dt=0) == E.KDA_ERR_UNSUPPORTED
 
@@ -119,6 +120,7 @@ def test_decode_host_validation(lib):
     assert call(ok, dk=100, dv=100) == binding.KDA_ERR_UNSUPPORTED
     assert call(ok, B=-1) == binding.KDA_ERR_INVALID_ARGUMENT
     assert call(ok, B=0) == binding.KDA_OK
+    assert call(ok, B=1 << 16, H=1 << 15) == binding.KDA_ERR_INVALID_ARGUMENT  # 2^31 units
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
