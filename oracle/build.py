@@ -1,6 +1,6 @@
 """Compile the fp64 C oracle into oracle/libkda_oracle.so.
 
-Test infrastructure only: this builds the checker that tests/, smoke() and the
+Test infrastructure only: this builds the oracle library that tests/, smoke() and the
 CPU-baseline leg of bench.py load; nothing in the product links it.
 """
 import os
