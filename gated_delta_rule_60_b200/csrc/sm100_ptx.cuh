@@ -261,34 +261,12 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, tf32 inputs (32-bit A columns)
-__device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// 32 lanes x 16 columns of 32 bit: thread i of the warp gets lane (base + i).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-          "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-          "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -303,14 +281,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-        "r"(r[7])
-        : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -344,39 +314,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// tf32 x tf32 -> f32 (kind::tf32), same field layout as idesc_bf16.
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn) {
-    return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn ? 1u : 0u) << 15) |
-           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// Byte offset of fp32 element (row, col) of a [rows][32] fp32 region in the
-// 128B-swizzled layout (32 elements per 128-byte row).
-__host__ __device__ __forceinline__ uint32_t sw128_off32(uint32_t row, uint32_t col) {
-    return (row >> 3) * 1024u + (row & 7u) * 128u +
-           ((((col >> 2) ^ (row & 7u)) & 7u) << 4) + (col & 3u) * 4u;
-}
-
-// Byte offset of fp32 element (row, k) of a [16][16] fp32 K-major tile in the
-// no-swizzle core-matrix layout (8 rows x 16 B cores) with LBO = 128 (next
-// 4 k) and SBO = 512 (next 8 rows).
-__host__ __device__ __forceinline__ uint32_t core16_off32(uint32_t row, uint32_t k) {
-    return (row >> 3) * 512u + (k >> 2) * 128u + (row & 7u) * 16u + (k & 3u) * 4u;
-}
-
 // Byte offset of element (row, col) of a [rows][64] bf16 region in the
 // 128B-swizzled layout (the TMA SWIZZLE_128B box layout and the canonical
 // K-major / MN-major 128B-swizzle atom).  The region must be 1024-aligned.
 __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t col) {
     return (row >> 3) * 1024u + (row & 7u) * 128u +
            ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + (col & 7u) * 2u;
-}
-
-// Byte offset of element (row, k) of a [16][16] bf16 K-major tile in the
-// no-swizzle core-matrix layout with LBO = 128 (next 8 k) and SBO = 256
-// (next 8 rows).
-__host__ __device__ __forceinline__ uint32_t core16_off(uint32_t row, uint32_t k) {
-    return (row >> 3) * 256u + (k >> 3) * 128u + (row & 7u) * 16u + (k & 7u) * 2u;
 }
 
 // Packed fp32 pair arithmetic (sm_100 f32x2 instructions).
