@@ -34,7 +34,8 @@
 // Everything that does not involve S0 (gate, decays, A_kk, A_qk, T, P, Z,
 // Ke, Qe) is prepared ahead of time.
 //
-// CTA = one (sequence, head) chain, 512 threads:
+// CTA = one (sequence, head) chain (a packed batch hands out its chains
+// longest first), 512 threads:
 //   warps 0-3   scan warpgroup: one thread per value channel; thread 0
 //               issues the step products, lane 0 of warp 1 the tile loads,
 //               lane 0 of warp 2 the L2 prefetches and the TMA stores of o
