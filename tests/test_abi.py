@@ -131,3 +131,22 @@ def test_binding_fails_loudly_without_library(tmp_path):
             binding.load_library(str(tmp_path / "missing.so"))
     finally:
         binding._lib = saved
+
+
+def test_binding_refuses_host_tensors(lib):
+    """No CPU path: host tensors are rejected before the library is called."""
+    import torch
+    T, H, d = 32, 2, 16
+    q = torch.zeros(T, H, d)
+    beta = torch.zeros(T, H)
+    with pytest.raises(ValueError, match="must be on"):
+        binding.kda_chunk_fwd(q, q, q, q, beta)
+    with pytest.raises(ValueError, match="must be on"):
+        binding.kda_decode_step(q[:2], q[:2], q[:2], q[:2], beta[:2],
+                                torch.zeros(2, H, d, d))
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(ImportError, match="not built"):
+        binding.load_library(str(tmp_path / "libkda.so"))
