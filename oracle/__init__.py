@@ -9,6 +9,9 @@ module only marshals numpy arrays through ctypes.  Every function takes the
 exact values the GPU receives, widened to fp64, so input rounding is not
 counted as kernel error.
 
+The steps just before and after the operator (short-conv prologue, output
+gate) are plain numpy in layer_ops.py.
+
 Recurrence, per head (pages: "Kimi K3 发布核实与 Moonshot AI 主干架构演变" §3
 "KDA 为什么不同于 MLA" and "K3 对 Kimi Linear 的进一步修改" bullet 1):
     a_t = exp(-5 * sigmoid(g_t));  S = Diag(a_t) S
@@ -20,6 +23,7 @@ import os
 import numpy as np
 
 from . import build as _build
+from .layer_ops import l2_normalize, output_gate, prologue, short_conv  # noqa: F401
 
 _lib = None
 
