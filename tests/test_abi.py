@@ -150,3 +150,18 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(ImportError, match="not built"):
         binding.load_library(str(tmp_path / "libkda.so"))
+
+
+def test_noalloc_refuses_oversized_scratch_on_the_host(lib):
+    """Scratch beyond the static 16 MiB array (the 1M-token, 16-head shape)
+    is refused before any device access; the pointers are never used."""
+    T, H = 1 << 20, 16
+    assert lib.kda_chunk_fwd_workspace_size(1, T, H, 128, 128, 0) > 16 << 20
+    P = ctypes.c_void_p
+    st = lib.kda_chunk_fwd_noalloc(P(256), P(256), P(256), P(256), P(256), None, None,
+                                   1, T, H, 128, 128, 0, P(256), None, None)
+    assert st == binding.KDA_ERR_WORKSPACE
+    # argument errors still win over the scratch check
+    st = lib.kda_chunk_fwd_noalloc(None, P(256), P(256), P(256), P(256), None, None,
+                                   1, T, H, 128, 128, 0, P(256), None, None)
+    assert st == binding.KDA_ERR_INVALID_ARGUMENT
