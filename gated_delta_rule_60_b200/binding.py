@@ -69,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_status_string.argtypes = [ctypes.c_int]
     lib.kda_version.restype = i32
     lib.kda_version.argtypes = []
+    lib.kda_selftest_wait_timeout.restype = ctypes.c_int
+    lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
     _lib = lib
     return lib
 
@@ -230,6 +232,14 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_step")
     return o
+
+
+def kda_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Let one bounded wait run out on the GPU (no fault): afterwards
+    kda_stream_status() reports KDA_ERR_TIMEOUT."""
+    st = load_library().kda_selftest_wait_timeout(int(limit_cycles), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_selftest_wait_timeout")
 
 
 def kda_stream_status(stream=None) -> int:

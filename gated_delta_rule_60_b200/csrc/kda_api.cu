@@ -200,3 +200,4 @@ kda_status kda_stream_status(void *stream) {
 }  // extern "C"
 
 #include "kda_noalloc.cuh"
+#include "kda_selftest.cuh"

@@ -166,6 +166,17 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const voi
  */
 KDA_API kda_status kda_stream_status(void *stream);
 
+/*
+ * Diagnostic of the failure-reporting path, with no fault: launches one tiny
+ * kernel on `stream` whose single thread waits, with the same bounded wait as
+ * the prefill pipeline, on a barrier that nothing ever arrives on.  After
+ * limit_cycles SM clock cycles (1 .. 2^32; about 0.5 ns each) the wait gives
+ * up and sets KDA_ERR_TIMEOUT in the status word, as a stalled pipeline stage
+ * would; kda_stream_status() then reports it and the context stays usable.
+ * Returns KDA_ERR_INVALID_ARGUMENT for a limit outside that range.
+ */
+KDA_API kda_status kda_selftest_wait_timeout(uint64_t limit_cycles, void *stream);
+
 /* Static English description of a status code (never NULL). */
 KDA_API const char *kda_status_string(kda_status s);
 

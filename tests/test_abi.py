@@ -165,3 +165,8 @@ def test_noalloc_refuses_oversized_scratch_on_the_host(lib):
     st = lib.kda_chunk_fwd_noalloc(None, P(256), P(256), P(256), P(256), None, None,
                                    1, T, H, 128, 128, 0, P(256), None, None)
     assert st == binding.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_selftest_limit_is_checked_on_the_host(lib):
+    assert lib.kda_selftest_wait_timeout(0, None) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_selftest_wait_timeout((1 << 32) + 1, None) == binding.KDA_ERR_INVALID_ARGUMENT
