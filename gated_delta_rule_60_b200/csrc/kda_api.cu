@@ -12,6 +12,8 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace {
 
 inline bool aligned16(const void *p) {
@@ -76,7 +78,10 @@ kda_status dispatch_decode(int d, const void *q, const void *k, const void *v,
     case 16: return launch_decode<T, 16, 1>(q, k, v, g, beta, S, o, units, s);
     case 32: return launch_decode<T, 32, 1>(q, k, v, g, beta, S, o, units, s);
     case 64: return launch_decode<T, 64, 1>(q, k, v, g, beta, S, o, units, s);
-    case 128: return launch_decode<T, 128, 2>(q, k, v, g, beta, S, o, units, s);
+    case 128:
+        kda::decode_step_d128_kernel<T><<<(unsigned)units, kda::kDecode128Threads, 0, s>>>(
+            (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta, S, (T *)o);
+        return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     default: return KDA_ERR_UNSUPPORTED;
     }
 }
@@ -182,16 +187,19 @@ KDA_API int kda_debug_cta_times(unsigned long long *dst, size_t n) {
 #endif
 
 kda_status kda_stream_status(void *stream) {
-    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return KDA_ERR_CUDA;
+    static std::atomic<unsigned> next_slot{0};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    // read and clear the word in one atomic exchange, on this stream
+    const int slot = (int)(next_slot.fetch_add(1u, std::memory_order_relaxed) % kda::kStatusSlots);
+    kda::status_take_kernel<<<1, 1, 0, s>>>(slot);
+    if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     unsigned int word = 0;
-    if (cudaMemcpyFromSymbol(&word, kda::g_status_word, sizeof(word)) != cudaSuccess)
+    if (cudaMemcpyFromSymbolAsync(&word, kda::g_status_taken, sizeof(word),
+                                  sizeof(word) * (size_t)slot, cudaMemcpyDeviceToHost,
+                                  s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
         return KDA_ERR_CUDA;
-    if (word != 0) {
-        const unsigned int zero = 0;
-        if (cudaMemcpyToSymbol(kda::g_status_word, &zero, sizeof(zero)) != cudaSuccess)
-            return KDA_ERR_CUDA;
-    }
     if (word & kda::kErrTimeout) return KDA_ERR_TIMEOUT;
     if (word & kda::kErrSeqlens) return KDA_ERR_BAD_SEQLENS;
     return KDA_OK;

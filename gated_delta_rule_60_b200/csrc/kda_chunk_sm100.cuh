@@ -55,6 +55,7 @@
 #include "sm100_ptx.cuh"
 #include "../../include/kda.h"
 
+#include <atomic>
 #include <cuda.h>
 
 namespace kda {
@@ -198,7 +199,11 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
         c.hT = (p.hT && c.ok) ? p.hT + unit * kSt : nullptr;
         return c;
     }
-    c.ok = true;
+    // One sequence per head, split into segments: its bounds must still be
+    // [0, T_tot).  Every CTA checks them before any access; a malformed
+    // cu_seqlens is reported and the CTA does nothing.
+    int64_t b0 = 0, b1 = 0;
+    c.ok = seq_bounds(p.cu, 0, 1, p.T_tot, b0, b1);
     int s;
     if (p.mode == kModeSegLocal && cta < p.H * p.G) {
         c.h = cta / p.G;
@@ -225,6 +230,11 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
     c.start = (int64_t)s * p.seg_len;
     const int64_t rem = p.T_tot - c.start;
     c.L = (int)(rem < p.seg_len ? rem : p.seg_len);
+    if (!c.ok) {
+        c.L = 0;
+        c.hT = nullptr;
+        c.write_o = false;
+    }
     return c;
 }
 
@@ -1011,15 +1021,19 @@ inline bool make_qkvg_map(CUtensorMap *map, const void *base, int H, int64_t T_t
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// SM count of the current device, looked up once per device.
 inline int sm_count() {
-    static int n = 0;
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cache[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    int n = (dev >= 0 && dev < kMaxDev) ? cache[dev].load(std::memory_order_relaxed) : 0;
     if (n == 0) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-            n = v;
-        else
-            n = 148;
+        int v = 0;
+        n = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0
+                ? v
+                : 148;
+        if (dev >= 0 && dev < kMaxDev) cache[dev].store(n, std::memory_order_relaxed);
     }
     return n;
 }
@@ -1063,10 +1077,14 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
                                   int64_t T_tot, int H, void *o, float *hT, void *workspace,
                                   cudaStream_t s) {
     CUtensorMap mq, mk, mv, mg, mo;
+    // With no tokens the token pointers may be NULL and no tile is ever
+    // copied (every chain is empty, or malformed and skipped); the maps then
+    // describe one row of hT, which the caller passes whenever this runs.
     const int64_t T_map = T_tot > 0 ? T_tot : 1;
-    if (!make_qkvg_map(&mq, q, H, T_map) || !make_qkvg_map(&mk, k, H, T_map) ||
-        !make_qkvg_map(&mv, v, H, T_map) || !make_qkvg_map(&mg, g, H, T_map) ||
-        !make_qkvg_map(&mo, o, H, T_map))
+    auto base = [&](const void *ptr) { return T_tot > 0 ? ptr : static_cast<const void *>(hT); };
+    if (!make_qkvg_map(&mq, base(q), H, T_map) || !make_qkvg_map(&mk, base(k), H, T_map) ||
+        !make_qkvg_map(&mv, base(v), H, T_map) || !make_qkvg_map(&mg, base(g), H, T_map) ||
+        !make_qkvg_map(&mo, base(o), H, T_map))
         return KDA_ERR_CUDA;
     auto kern = prefill::chunk_fwd_sm100_kernel;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

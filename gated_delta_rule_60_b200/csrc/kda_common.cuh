@@ -16,6 +16,16 @@ namespace kda {
 enum : unsigned { kErrSeqlens = 1u, kErrTimeout = 2u };
 __device__ unsigned int g_status_word;
 
+// kda_stream_status() takes the word with one atomic exchange on the device,
+// so a bit set by a kernel on another stream is never lost between a read
+// and a clear.  Each call gets its own slot for the value it took.
+constexpr int kStatusSlots = 64;
+__device__ unsigned int g_status_taken[kStatusSlots];
+
+__global__ void status_take_kernel(int slot) {
+    g_status_taken[slot] = atomicExch(&g_status_word, 0u);
+}
+
 __device__ __forceinline__ void raise_error(unsigned bit) {
     atomicOr(&g_status_word, bit);
 }

@@ -14,7 +14,8 @@
 // SPLIT row parts through shared memory, then every part writes its rows back.
 // Each state element is read once and written once, with the streaming
 // (evict-first) cache hint: the state is far larger than L2 and is not
-// re-read within a step.
+// re-read within a step.  d = 128 has its own kernel below with 128-bit
+// accesses.
 #pragma once
 
 #include "kda_common.cuh"
@@ -93,6 +94,91 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
 #pragma unroll
         for (int i = 0; i < R; ++i)
             __stcs(Su + (size_t)i * D, fmaf(sk[hl][part * R + i], uj, s[i]));
+    }
+}
+
+// d = 128: the state of one (b, h) is 128 rows of 512 bytes.  Warp w of the
+// 256-thread block owns rows 16 w .. 16 w + 15; lane l owns columns
+// 4 l .. 4 l + 3 of each, so every access is one 128-bit streaming load or
+// store and a warp covers a whole row in one instruction.  A thread issues its
+// 16 row loads back to back (64 KB in flight per block) before it needs any
+// of them.  The column sums r = S'^T k and p = S'^T q are partial per warp and
+// meet in shared memory.
+__device__ __forceinline__ float4 ld_stream_f4(const float *p) {
+    float4 r;
+    asm volatile("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_stream_f4(float *p, float4 v) {
+    asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+constexpr int kDecode128Threads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kDecode128Threads)
+decode_step_d128_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                        const T *__restrict__ v, const T *__restrict__ g,
+                        const T *__restrict__ beta, float *__restrict__ S,
+                        T *__restrict__ o) {
+    constexpr int D = 128, W = kDecode128Threads / 32, R = D / W;
+    __shared__ float sa[D], sk[D], sq[D], su[D];
+    __shared__ float4 sr[W][D / 4], sp[W][D / 4];
+    const long u = blockIdx.x;
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    float *Su = S + (size_t)u * D * D + (size_t)(R * w) * D + 4 * l;
+    float4 s[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) s[i] = ld_stream_f4(Su + (size_t)i * D);
+    if (tid < D) {
+        const size_t e = (size_t)u * D + tid;
+        sq[tid] = IO<T>::ld(q + e);
+        sk[tid] = IO<T>::ld(k + e);
+        sa[tid] = expf(log_decay(IO<T>::ld(g + e)));
+    }
+    __syncthreads();
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int row = R * w + i;
+        const float a = sa[row], kr = sk[row], qr = sq[row];
+        s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+        r.x = fmaf(s[i].x, kr, r.x); r.y = fmaf(s[i].y, kr, r.y);
+        r.z = fmaf(s[i].z, kr, r.z); r.w = fmaf(s[i].w, kr, r.w);
+        p.x = fmaf(s[i].x, qr, p.x); p.y = fmaf(s[i].y, qr, p.y);
+        p.z = fmaf(s[i].z, qr, p.z); p.w = fmaf(s[i].w, qr, p.w);
+    }
+    sr[w][l] = r;
+    sp[w][l] = p;
+    __syncthreads();
+    if (tid < D) {
+        const int j = tid;
+        float kq = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) kq = fmaf(sk[i], sq[i], kq);
+        const float *srf = reinterpret_cast<const float *>(sr);
+        const float *spf = reinterpret_cast<const float *>(sp);
+        float rj = 0.f, pj = 0.f;
+#pragma unroll
+        for (int x = 0; x < W; ++x) { rj += srf[x * D + j]; pj += spf[x * D + j]; }
+        const float uj = IO<T>::ld(beta + u) * (IO<T>::ld(v + (size_t)u * D + j) - rj);
+        su[j] = uj;
+        IO<T>::st(o + (size_t)u * D + j, fmaf(uj, kq, pj));
+    }
+    __syncthreads();
+    const float4 uu = reinterpret_cast<const float4 *>(su)[l];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const float kr = sk[R * w + i];
+        float4 y = s[i];
+        y.x = fmaf(kr, uu.x, y.x); y.y = fmaf(kr, uu.y, y.y);
+        y.z = fmaf(kr, uu.z, y.z); y.w = fmaf(kr, uu.w, y.w);
+        st_stream_f4(Su + (size_t)i * D, y);
     }
 }
 

@@ -162,7 +162,11 @@ KDA_API kda_status kda_chunk_fwd_noalloc(const void *q, const void *k, const voi
 /*
  * Synchronises `stream`, then returns and clears the current device's
  * status word: KDA_OK, KDA_ERR_TIMEOUT, KDA_ERR_BAD_SEQLENS, or
- * KDA_ERR_CUDA if the synchronisation itself failed.
+ * KDA_ERR_CUDA if the synchronisation itself failed.  The word is per
+ * device, not per stream: a bit may come from a kernel on another stream of
+ * the same device.  It is read and cleared in one atomic exchange (a one-
+ * thread kernel on `stream`), so no bit raised meanwhile is lost; it is then
+ * reported by the next call.
  */
 KDA_API kda_status kda_stream_status(void *stream);
 

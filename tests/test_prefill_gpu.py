@@ -1,6 +1,8 @@
 """GPU parity of kda_chunk_fwd against the fp64 oracle, plus metamorphic
 properties that need no oracle (split-carry, varlen packing, determinism,
 no-op padding, decode = prefill)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -241,3 +243,36 @@ def test_long_1m_workload_sampled():
     mask = np.zeros((1, w.H), dtype=bool)
     mask[0, np.random.default_rng(3).choice(w.H, 2, replace=False)] = True
     check(inp, o, hT, unit_mask=mask)
+
+
+@pytest.mark.parametrize("with_h0", [True, False])
+def test_all_empty_batch_writes_hT(with_h0):
+    """No tokens at all but a final state asked for: the token pointers may be
+    NULL, and hT must be h0 (or zero) for every (sequence, head)."""
+    N, H, d = 3, 2, 128
+    h0 = torch.randn(N, H, d, d, device="cuda") if with_h0 else None
+    hT = torch.full((N, H, d, d), 7.0, device="cuda")
+    cu = torch.zeros(N + 1, dtype=torch.int32, device="cuda")
+    lib = binding.load_library()
+    P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    st = lib.kda_chunk_fwd(None, None, None, None, None, P(h0), P(cu), N, 0, H, d, d,
+                           binding.KDA_BF16, None, P(hT), None, 0, None)
+    assert st == binding.KDA_OK
+    assert binding.kda_stream_status() == binding.KDA_OK
+    assert torch.equal(hT, h0 if with_h0 else torch.zeros_like(hT))
+
+
+def test_bad_seqlens_on_the_segmented_path():
+    """One long sequence per head runs split into segments; a cu_seqlens whose
+    last entry is not T_tot must still be reported, with nothing written."""
+    T, H = 16384 + 77, 2
+    assert binding.kda_chunk_fwd_workspace_size(1, T, H, 128, 128, torch.bfloat16) > 0
+    inp = inputs.make_prefill([T], H, 128, 128, torch.bfloat16, seed=98)
+    d = to_device(inp)
+    bad = torch.tensor([0, T - 1], dtype=torch.int32, device="cuda")
+    o = torch.zeros(T, H, 128, dtype=torch.bfloat16, device="cuda")
+    hT = torch.zeros(1, H, 128, 128, dtype=torch.float32, device="cuda")
+    binding.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, bad, o=o, hT=hT)
+    assert binding.kda_stream_status() == binding.KDA_ERR_BAD_SEQLENS
+    assert binding.kda_stream_status() == binding.KDA_OK
+    assert int(torch.count_nonzero(o)) == 0 and int(torch.count_nonzero(hT)) == 0
