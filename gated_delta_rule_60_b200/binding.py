@@ -71,6 +71,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_version.argtypes = []
     lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.kda_debug_stall_prefill.restype = ctypes.c_int
+    lib.kda_debug_stall_prefill.argtypes = [i32, ctypes.c_uint64]
     _lib = lib
     return lib
 
@@ -240,6 +242,15 @@ def kda_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
     st = load_library().kda_selftest_wait_timeout(int(limit_cycles), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_selftest_wait_timeout")
+
+
+def kda_debug_stall_prefill(step: int, limit_cycles: int) -> None:
+    """Make the next tensor-core kda_chunk_fwd call stall its scan at state
+    step `step` on a wait that nothing completes, bounded by limit_cycles
+    (no fault: the kernel reports KDA_ERR_TIMEOUT, drains and returns)."""
+    st = load_library().kda_debug_stall_prefill(int(step), int(limit_cycles))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_debug_stall_prefill")
 
 
 def kda_stream_status(stream=None) -> int:

@@ -186,6 +186,15 @@ KDA_API int kda_debug_cta_times(unsigned long long *dst, size_t n) {
 }
 #endif
 
+kda_status kda_debug_stall_prefill(int32_t step, uint64_t limit_cycles) {
+    if (step < 0 || limit_cycles == 0 || limit_cycles > (1ull << 32))
+        return KDA_ERR_INVALID_ARGUMENT;
+    kda::DebugStall &d = kda::debug_stall();
+    d.limit.store((unsigned long long)limit_cycles);
+    d.step.store(step);
+    return KDA_OK;
+}
+
 kda_status kda_stream_status(void *stream) {
     static std::atomic<unsigned> next_slot{0};
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

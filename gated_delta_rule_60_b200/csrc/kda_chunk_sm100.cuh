@@ -136,6 +136,7 @@ struct Barriers {
     uint64_t a_done[kPrep], z_done[kPrep], b_ready[kPrep];
     uint64_t mma1_done, d_done;
     uint64_t drain_scan, drain_prep[kPrep];
+    uint64_t never;                  // diagnostic: a barrier nothing arrives on
     float beta_s[kPrep][kStep];
     int stop[kPrep + 1];             // per-warpgroup exit decision (last: scan)
     uint32_t tmem_base;
@@ -165,6 +166,8 @@ struct Params {
     int mode, G;
     long seg_len;
     float *ws_R, *ws_M, *ws_S;    // [G][H][128][128] each (segment modes)
+    unsigned long long wait_limit;  // bound of a pipeline wait, SM clock cycles
+    int stall_step;               // diagnostic: step at which the scan waits on `never` (-1: none)
 };
 
 // What one CTA runs: a token range of one head, where its state starts and
@@ -296,9 +299,9 @@ __device__ __forceinline__ float2 decay2(float2 g) {
 
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort) {
+                                          volatile int *abort, unsigned long long limit) {
     bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, kWaitLimit);
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     return ok;
 }
@@ -413,6 +416,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             bars.stop[i] = 0;
         }
         mbar_init(&bars.mma1_done, 1);
+        mbar_init(&bars.never, 1);
         mbar_init(&bars.d_done, 1);
         mbar_init(&bars.drain_scan, 1);
         bars.stop[kPrep] = 0;
@@ -482,7 +486,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         bool alive = nS > 0;
         if (alive) {
             // initial state: gamma_0 * S0 (fp32) and bf16(S0)
-            if (warp_wait(&bars.b_ready[0], 0, abortp)) {
+            if (warp_wait(&bars.b_ready[0], 0, abortp, p.wait_limit)) {
                 const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA);
 #pragma unroll 1
                 for (int part = 0; part < 4; ++part) {
@@ -571,6 +575,9 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         for (int c = 0; alive && c < nS; ++c) {
             const int sl = c % kSlots;
             const uint32_t slot_u = s_base + SM_SLOT + sl * kSlotBytes;
+            // diagnostic: a wait that nothing completes, so that the bounded
+            // wait runs out here and the CTA takes its abort and drain path
+            if (c == p.stall_step && !warp_wait(&bars.never, 0, abortp, p.wait_limit)) fail(bars);
             // ---- MMA1: [(Ke S)^T | (Qe S)^T] = bf16(S)^T [Ke ; Qe]^T, then the v part of MMA2
             if (tid == 0 && !*abortp) {
                 KDA_TR(TR_SCAN_ISSUE, c);
@@ -596,7 +603,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             if (loader && c >= 1 && c - 1 + kSlots < nS && !*abortp) load_step(c - 1 + kSlots);
             if (prefetcher && c >= 1 && c - 1 + 2 * kSlots < nS) prefetch_step(c - 1 + 2 * kSlots);
             // ---- -(Ke S)^T in bf16: A operand of the second half of MMA2
-            if (warp_wait(&bars.mma1_done, c & 1, abortp)) {
+            if (warp_wait(&bars.mma1_done, c & 1, abortp, p.wait_limit)) {
                 if (tid == 0) KDA_TR(TR_S_M1, c);
                 tc_fence_after();
                 uint32_t u[32], un[16];
@@ -628,12 +635,12 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             store_o();                      // outputs of step c - 1, during the MMA2 round trip
             // ---- step done: outputs, next step's operands (or the final state)
-            if (warp_wait(&bars.d_done, c & 1, abortp)) {
+            if (warp_wait(&bars.d_done, c & 1, abortp, p.wait_limit)) {
                 tc_fence_after();
                 if (tid == 0) KDA_TR(TR_SCAN_DONE, c);
                 const bool has_next = c + 1 < nS;
                 bool ready = true;
-                if (has_next) ready = warp_wait(&bars.b_ready[(c + 1) % kPrep], ((c + 1) / kPrep) & 1, abortp);
+                if (has_next) ready = warp_wait(&bars.b_ready[(c + 1) % kPrep], ((c + 1) / kPrep) & 1, abortp, p.wait_limit);
                 if (!ready) fail(bars);
                 if (tid == 0) KDA_TR(TR_S_BR, c);
                 const int sn = (c + 1) % kSlots;
@@ -743,7 +750,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 bars.beta_s[pg][lane] = beta_pre;
                 if (s + kPrep < nS) beta_pre = load_beta(s + kPrep);
             }
-            bool ok = warp_wait(&bars.slot_full[sl], (s / kSlots) & 1, abortp);
+            bool ok = warp_wait(&bars.slot_full[sl], (s / kSlots) & 1, abortp, p.wait_limit);
             if (!ok) fail(bars);
             if (ok && pt == 0) KDA_TR(TR_PREP_FULL, s);
 
@@ -780,7 +787,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
             } else {
                 // warp 0: (Diag(beta) strict_lower(A_kk))^T; warp 1: causal(A_qk)
-                if (warp_wait(&bars.a_done[pg], par, abortp)) {
+                if (warp_wait(&bars.a_done[pg], par, abortp, p.wait_limit)) {
                     if (pt == 0) KDA_TR(TR_PREP_A, s);
                     tc_fence_after();
                     uint32_t d[32];
@@ -883,7 +890,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
             }
             // ---------------- [P ; Diag(delta) Z]: operand B of MMA2
-            if (warp_wait(&bars.z_done[pg], par, abortp)) {
+            if (warp_wait(&bars.z_done[pg], par, abortp, p.wait_limit)) {
                 if (pt == 0) KDA_TR(TR_PREP_Z, s);
                 tc_fence_after();
                 uint32_t zv[32];
@@ -1066,6 +1073,18 @@ inline SegPlan plan_segments(int N, int64_t T, int H) {
     return pl;
 }
 
+// One-shot diagnostic (kda_debug_stall_prefill): the next tensor-core
+// prefill call makes every CTA's scan wait, at step `step`, on a barrier that
+// nothing arrives on, with a bound of `limit` cycles.
+struct DebugStall {
+    std::atomic<int> step{-1};
+    std::atomic<unsigned long long> limit{0};
+};
+inline DebugStall &debug_stall() {
+    static DebugStall d;
+    return d;
+}
+
 inline size_t sm100_workspace_bytes(int N, int64_t T, int H) {
     const SegPlan pl = plan_segments(N, T, H);
     if (pl.G <= 1) return 0;
@@ -1103,6 +1122,9 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.G = 1;
     p.seg_len = (long)T_tot;
     p.ws_R = p.ws_M = p.ws_S = nullptr;
+    p.stall_step = debug_stall().step.exchange(-1);
+    const unsigned long long lim = debug_stall().limit.exchange(0);
+    p.wait_limit = (p.stall_step >= 0 && lim > 0) ? lim : prefill::kWaitLimit;
     const SegPlan pl = plan_segments(N, T_tot, H);
     if (pl.G <= 1) {
         kern<<<(unsigned)(N * H), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);

@@ -181,6 +181,22 @@ KDA_API kda_status kda_stream_status(void *stream);
  */
 KDA_API kda_status kda_selftest_wait_timeout(uint64_t limit_cycles, void *stream);
 
+/*
+ * Diagnostic of the prefill pipeline's own failure path, with no fault: the
+ * NEXT kda_chunk_fwd call that runs the tensor-core path (KDA_BF16,
+ * dk = dv = 128) makes the scan of every CTA wait, at state step `step`
+ * (32 tokens each), on a barrier that nothing ever arrives on, and bounds
+ * every pipeline wait of that call by limit_cycles SM clock cycles.  The
+ * wait gives up, the kernel sets KDA_ERR_TIMEOUT in the status word, every
+ * role of the CTA leaves its loop, the CTA waits for its own copies, stores
+ * and tensor-core products, frees its tensor memory and returns; nothing is
+ * written outside o and hT.  The values of that call's outputs are then
+ * undefined.  The setting is consumed by that one call (process-wide, not
+ * per device or stream).  Returns KDA_ERR_INVALID_ARGUMENT for step < 0 or a
+ * limit outside 1 .. 2^32.
+ */
+KDA_API kda_status kda_debug_stall_prefill(int32_t step, uint64_t limit_cycles);
+
 /* Static English description of a status code (never NULL). */
 KDA_API const char *kda_status_string(kda_status s);
 

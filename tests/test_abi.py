@@ -170,3 +170,10 @@ def test_noalloc_refuses_oversized_scratch_on_the_host(lib):
 def test_selftest_limit_is_checked_on_the_host(lib):
     assert lib.kda_selftest_wait_timeout(0, None) == binding.KDA_ERR_INVALID_ARGUMENT
     assert lib.kda_selftest_wait_timeout((1 << 32) + 1, None) == binding.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_prefill_stall_diagnostic_checks_its_arguments(lib):
+    """Invalid requests are refused on the host and arm nothing."""
+    assert lib.kda_debug_stall_prefill(-1, 1000) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_debug_stall_prefill(0, 0) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_debug_stall_prefill(0, (1 << 32) + 1) == binding.KDA_ERR_INVALID_ARGUMENT
