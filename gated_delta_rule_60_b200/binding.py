@@ -57,6 +57,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                   i32, ctypes.c_int, vp, vp, vp, sz, vp]
+    lib.kda_chunk_fwd_gated.restype = ctypes.c_int
+    lib.kda_chunk_fwd_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                        i32, ctypes.c_int, vp, vp, vp, vp, sz, vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                           i32, ctypes.c_int, vp, vp, vp]
@@ -71,6 +74,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_version.argtypes = []
     lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.kda_prologue.restype = ctypes.c_int
+    lib.kda_prologue.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                 ctypes.c_int, vp, vp, vp, vp, vp]
     lib.kda_debug_stall_prefill.restype = ctypes.c_int
     lib.kda_debug_stall_prefill.argtypes = [i32, ctypes.c_uint64]
     _lib = lib
@@ -169,6 +175,56 @@ def kda_chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return o, hT
 
 
+def kda_chunk_fwd_gated(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        g: torch.Tensor, beta: torch.Tensor, z: torch.Tensor,
+                        h0: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None, *,
+                        num_seqs: Optional[int] = None,
+                        o: Optional[torch.Tensor] = None,
+                        hT: Optional[torch.Tensor] = None,
+                        output_final_state: bool = True,
+                        workspace: Optional[torch.Tensor] = None,
+                        stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_chunk_fwd with the output gate fused into the output store:
+    o = (S^T q) * sigmoid(z), z [T_tot, H, dv] in the inputs' dtype."""
+    lib = load_library()
+    dev = q.device
+    T_tot, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name, shp in ((q, "q", (T_tot, H, dk)), (k, "k", (T_tot, H, dk)),
+                         (g, "g", (T_tot, H, dk)), (v, "v", (T_tot, H, dv)),
+                         (beta, "beta", (T_tot, H)), (z, "z", (T_tot, H, dv))):
+        _check(t, name, dt, shp, dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty(T_tot, H, dv, dtype=dt, device=dev)
+    _check(o, "o", dt, (T_tot, H, dv), dev)
+    if hT is None and output_final_state:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    ws_need = kda_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dt)
+    if ws_need and workspace is None:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kda_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(h0), _ptr(cu_seqlens), N, T_tot, H, dk, dv,
+                                 _DTYPES[dt], _ptr(z), _ptr(o), _ptr(hT), _ptr(workspace),
+                                 ws_bytes, _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_gated")
+    return o, hT
+
+
 def kda_chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                           g: torch.Tensor, beta: torch.Tensor,
                           h0: Optional[torch.Tensor] = None,
@@ -242,6 +298,40 @@ def kda_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
     st = load_library().kda_selftest_wait_timeout(int(limit_cycles), _stream_handle(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_selftest_wait_timeout")
+
+
+def kda_prologue(xq: torch.Tensor, xk: torch.Tensor, xv: torch.Tensor,
+                 wq: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor,
+                 beta_raw: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None, *,
+                 num_seqs: Optional[int] = None,
+                 stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Short-conv prologue: (q, k, v, beta) for kda_chunk_fwd from the raw
+    projections xq, xk, xv [T_tot, H, d], taps w* [H, d, 4] fp32 and
+    beta_raw [T_tot, H] (see include/kda.h)."""
+    lib = load_library()
+    dev = xq.device
+    T_tot, H, d = xq.shape
+    dt = xq.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name in ((xq, "xq"), (xk, "xk"), (xv, "xv")):
+        _check(t, name, dt, (T_tot, H, d), dev)
+    for t, name in ((wq, "wq"), (wk, "wk"), (wv, "wv")):
+        _check(t, name, torch.float32, (H, d, 4), dev)
+    _check(beta_raw, "beta_raw", dt, (T_tot, H), dev)
+    q, k, v = (torch.empty(T_tot, H, d, dtype=dt, device=dev) for _ in range(3))
+    beta = torch.empty(T_tot, H, dtype=dt, device=dev)
+    st = lib.kda_prologue(_ptr(xq), _ptr(xk), _ptr(xv), _ptr(wq), _ptr(wk), _ptr(wv),
+                          _ptr(beta_raw), _ptr(cu_seqlens), N, T_tot, H, d, _DTYPES[dt],
+                          _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prologue")
+    return q, k, v, beta
 
 
 def kda_debug_stall_prefill(step: int, limit_cycles: int) -> None:

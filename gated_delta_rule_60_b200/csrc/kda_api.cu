@@ -9,6 +9,7 @@
 #include "kda_decode.cuh"
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_sm100.cuh"
+#include "kda_prologue.cuh"
 
 #include <cuda_runtime.h>
 
@@ -32,7 +33,7 @@ template <typename T, int D>
 kda_status launch_simt(const void *q, const void *k, const void *v,
                        const void *g, const void *beta, const float *h0,
                        const int32_t *cu, int N, int64_t T_tot, int H,
-                       void *o, float *hT, cudaStream_t s) {
+                       const void *z, void *o, float *hT, cudaStream_t s) {
     const size_t smem = sizeof(kda::SimtSmem<D>);
     auto kern = kda::chunk_fwd_simt_kernel<T, D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -40,7 +41,7 @@ kda_status launch_simt(const void *q, const void *k, const void *v,
         return KDA_ERR_CUDA;
     kern<<<(unsigned)(N * H), 256, smem, s>>>(
         (const T *)q, (const T *)k, (const T *)v, (const T *)g,
-        (const T *)beta, h0, cu, N, (long)T_tot, H, (T *)o, hT);
+        (const T *)beta, h0, cu, N, (long)T_tot, H, (const T *)z, (T *)o, hT);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -48,12 +49,40 @@ template <typename T>
 kda_status dispatch_simt(int d, const void *q, const void *k, const void *v,
                          const void *g, const void *beta, const float *h0,
                          const int32_t *cu, int N, int64_t T_tot, int H,
-                         void *o, float *hT, cudaStream_t s) {
+                         const void *z, void *o, float *hT, cudaStream_t s) {
     switch (d) {
-    case 16: return launch_simt<T, 16>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
-    case 32: return launch_simt<T, 32>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
-    case 64: return launch_simt<T, 64>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
-    case 128: return launch_simt<T, 128>(q, k, v, g, beta, h0, cu, N, T_tot, H, o, hT, s);
+    case 16: return launch_simt<T, 16>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 32: return launch_simt<T, 32>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 64: return launch_simt<T, 64>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 128: return launch_simt<T, 128>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    default: return KDA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int D>
+kda_status launch_prologue(const void *xq, const void *xk, const void *xv, const float *wq,
+                           const float *wk, const float *wv, const void *braw, const int32_t *cu,
+                           int N, int64_t T_tot, int H, void *q, void *k, void *v, void *beta,
+                           cudaStream_t s) {
+    using Sh = kda::pro::Shape<D>;
+    const int64_t blocks = (T_tot + Sh::kTokPerBlock - 1) / Sh::kTokPerBlock;
+    const dim3 grid((unsigned)blocks, (unsigned)H, 3);
+    kda::pro::prologue_kernel<T, D><<<grid, kda::pro::kThreads, 0, s>>>(
+        (const T *)xq, (const T *)xk, (const T *)xv, wq, wk, wv, (const T *)braw, cu, N, T_tot, H,
+        (T *)q, (T *)k, (T *)v, (T *)beta);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <typename T>
+kda_status dispatch_prologue(int d, const void *xq, const void *xk, const void *xv,
+                             const float *wq, const float *wk, const float *wv, const void *braw,
+                             const int32_t *cu, int N, int64_t T_tot, int H, void *q, void *k,
+                             void *v, void *beta, cudaStream_t s) {
+    switch (d) {
+    case 16: return launch_prologue<T, 16>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
+    case 32: return launch_prologue<T, 32>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
+    case 64: return launch_prologue<T, 64>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
+    case 128: return launch_prologue<T, 128>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
     default: return KDA_ERR_UNSUPPORTED;
     }
 }
@@ -113,12 +142,12 @@ size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t T_tot, int32_t H,
     return 0;
 }
 
-kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
-                         const void *g, const void *beta, const float *h0,
-                         const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
-                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
-                         void *o, float *hT, void *workspace,
-                         size_t workspace_bytes, void *stream) {
+static kda_status chunk_fwd_impl(const void *q, const void *k, const void *v,
+                                 const void *g, const void *beta, const float *h0,
+                                 const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                                 int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                 const void *z, void *o, float *hT, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
     if (N < 0 || T_tot < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
     if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
     if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
@@ -131,6 +160,7 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
         const void *req[] = {q, k, v, g, beta, o};
         for (const void *p : req)
             if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+        if (z && !aligned16(z)) return KDA_ERR_INVALID_ARGUMENT;
     }
     if ((h0 && !aligned16(h0)) || (hT && !aligned16(hT)) ||
         (cu_seqlens && !aligned16(cu_seqlens)))
@@ -145,12 +175,33 @@ kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
         return T_tot == 0 && hT == nullptr
                    ? KDA_OK
                    : kda::sm100_chunk_fwd(q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H,
-                                          o, hT, workspace, s);
+                                          z, o, hT, workspace, s);
     if (dt == KDA_BF16)
         return dispatch_simt<__nv_bfloat16>(dk, q, k, v, g, beta, h0, cu_seqlens,
-                                            N, T_tot, H, o, hT, s);
+                                            N, T_tot, H, z, o, hT, s);
     return dispatch_simt<float>(dk, q, k, v, g, beta, h0, cu_seqlens, N, T_tot,
-                                H, o, hT, s);
+                                H, z, o, hT, s);
+}
+
+kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
+                         const void *g, const void *beta, const float *h0,
+                         const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                         void *o, float *hT, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H, dk, dv, dt, nullptr,
+                          o, hT, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
+                               const void *g, const void *beta, const float *h0,
+                               const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                               int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                               const void *z, void *o, float *hT, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    if (T_tot > 0 && z == nullptr) return KDA_ERR_INVALID_ARGUMENT;
+    return chunk_fwd_impl(q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H, dk, dv, dt, z, o, hT,
+                          workspace, workspace_bytes, stream);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v,
@@ -170,6 +221,28 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
     if (dt == KDA_BF16)
         return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, units, s);
     return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, units, s);
+}
+
+kda_status kda_prologue(const void *xq, const void *xk, const void *xv, const float *wq,
+                        const float *wk, const float *wv, const void *beta_raw,
+                        const int32_t *cu_seqlens, int32_t N, int64_t T_tot, int32_t H, int32_t d,
+                        kda_dtype dt, void *q, void *k, void *v, void *beta, void *stream) {
+    if (N < 0 || T_tot < 0 || H <= 0 || H > 65535) return KDA_ERR_INVALID_ARGUMENT;
+    if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
+    if (!supported_simt_d(d)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return T_tot == 0 ? KDA_OK : KDA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens == nullptr && (T_tot % N) != 0) return KDA_ERR_INVALID_ARGUMENT;
+    if (T_tot == 0) return KDA_OK;
+    const void *req[] = {xq, xk, xv, wq, wk, wv, beta_raw, q, k, v, beta};
+    for (const void *p : req)
+        if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens && !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == KDA_BF16)
+        return dispatch_prologue<__nv_bfloat16>(d, xq, xk, xv, wq, wk, wv, beta_raw, cu_seqlens, N,
+                                                T_tot, H, q, k, v, beta, s);
+    return dispatch_prologue<float>(d, xq, xk, xv, wq, wk, wv, beta_raw, cu_seqlens, N, T_tot, H,
+                                    q, k, v, beta, s);
 }
 
 #ifdef KDA_TRACE

@@ -19,7 +19,8 @@
 // (k = q = v = 0, beta = 0, log-decay 0).
 //
 // One CTA runs one (sequence, head) chain over all of its chunks; the state
-// lives in shared memory in fp32.
+// lives in shared memory in fp32.  With z given, every output row is
+// multiplied by sigmoid(z) before it is stored (the fused output gate).
 #pragma once
 
 #include "kda_common.cuh"
@@ -46,7 +47,7 @@ chunk_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, const T *__restrict__ g,
                       const T *__restrict__ beta, const float *__restrict__ h0,
                       const int32_t *__restrict__ cu, int N, long T_tot, int H,
-                      T *__restrict__ o, float *__restrict__ hT) {
+                      const T *__restrict__ z, T *__restrict__ o, float *__restrict__ hT) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem<D> &sm = *reinterpret_cast<SimtSmem<D> *>(smem_raw);
     const int tid = threadIdx.x;
@@ -153,7 +154,9 @@ chunk_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
             for (int c = 0; c < D; ++c) acc = fmaf(sm.Qa[r][c], sm.S[c][j], acc);
 #pragma unroll
             for (int i = 0; i < kChunk; ++i) acc = fmaf(sm.M[r][i], sm.U[i][j], acc);
-            IO<T>::st(o + ((size_t)(c0 + r) * H + h) * D + j, acc);
+            const size_t oe = ((size_t)(c0 + r) * H + h) * D + j;
+            if (z) acc *= out_gate(IO<T>::ld(z + oe));       // fused output gate
+            IO<T>::st(o + oe, acc);
         }
         __syncthreads();
         // 8. S = Diag(gamma) S0 + (K * e^{b_C - b})^T U

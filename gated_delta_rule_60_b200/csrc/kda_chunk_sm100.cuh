@@ -157,6 +157,7 @@ enum { kModeChains = 0, kModeSegLocal = 1, kModeSegFinal = 2 };
 
 struct Params {
     const __nv_bfloat16 *beta;
+    const __nv_bfloat16 *z;       // output gate: o * sigmoid(z), or NULL
     const float *h0;
     const int32_t *cu;
     __nv_bfloat16 *o;
@@ -374,6 +375,9 @@ __device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane,
     }
 }
 
+// kGate: the fused output gate o * sigmoid(z) (p.z), compiled only into the
+// gated instantiation so that the plain operator carries no trace of it.
+template <bool kGate>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
@@ -537,6 +541,16 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         auto store_o = [&]() {
             if (o_step < 0 || !ch.write_o) { o_step = -1; return; }
             const int Lc = L - kStep * o_step;
+            if (kGate) {
+                // fused output gate: o * sigmoid(z) on the values in registers
+                const __nv_bfloat16 *zr = p.z + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
+                const size_t step = (size_t)p.H * kD;
+#pragma unroll
+                for (int r = 0; r < kStep; ++r)
+                    if (r < Lc)
+                        ov[r] = __float_as_uint(__uint_as_float(ov[r]) *
+                                                out_gate(__bfloat162float(zr[(size_t)r * step])));
+            }
             if (Lc >= kStep) {
                 // lanes j, j ^ 1 swap half of their tokens so that each writes
                 // 32-bit words (channels j & ~1, j | 1) of 16 tokens
@@ -1093,8 +1107,8 @@ inline size_t sm100_workspace_bytes(int N, int64_t T, int H) {
 
 inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
                                   const void *beta, const float *h0, const int32_t *cu, int N,
-                                  int64_t T_tot, int H, void *o, float *hT, void *workspace,
-                                  cudaStream_t s) {
+                                  int64_t T_tot, int H, const void *z, void *o, float *hT,
+                                  void *workspace, cudaStream_t s) {
     CUtensorMap mq, mk, mv, mg, mo;
     // With no tokens the token pointers may be NULL and no tile is ever
     // copied (every chain is empty, or malformed and skipped); the maps then
@@ -1105,12 +1119,13 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
         !make_qkvg_map(&mv, base(v), H, T_map) || !make_qkvg_map(&mg, base(g), H, T_map) ||
         !make_qkvg_map(&mo, base(o), H, T_map))
         return KDA_ERR_CUDA;
-    auto kern = prefill::chunk_fwd_sm100_kernel;
+    auto kern = z ? prefill::chunk_fwd_sm100_kernel<true> : prefill::chunk_fwd_sm100_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)prefill::kSmemAlloc) != cudaSuccess)
         return KDA_ERR_CUDA;
     prefill::Params p;
     p.beta = static_cast<const __nv_bfloat16 *>(beta);
+    p.z = static_cast<const __nv_bfloat16 *>(z);
     p.h0 = h0;
     p.cu = cu;
     p.o = static_cast<__nv_bfloat16 *>(o);

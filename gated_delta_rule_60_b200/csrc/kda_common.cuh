@@ -39,6 +39,13 @@ __device__ __forceinline__ float log_decay(float g) {
     return -5.0f / (1.0f + e);
 }
 
+// Output gate o * sigmoid(z) (page "Kimi K3 发布核实与 Moonshot AI 主干架构演变",
+// §3 "K3 对 Kimi Linear 的进一步修改", bullet 2: a full-rank, input-dependent
+// channel gate on the output).  z = -inf gives 0, z = +inf gives 1.
+__device__ __forceinline__ float out_gate(float z) {
+    return 1.0f / (1.0f + __expf(-z));
+}
+
 template <typename T>
 struct IO;
 

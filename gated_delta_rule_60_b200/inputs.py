@@ -109,3 +109,34 @@ def make_state(B: int, H: int, dk: int, dv: int, std: float, seed: int
                ) -> torch.Tensor:
     gen = torch.Generator().manual_seed(int(seed))
     return torch.randn(B, H, dk, dv, generator=gen) * float(std)
+
+
+@dataclass
+class LayerInputs:
+    """Raw projections of a KDA layer (before the short-conv prologue)."""
+    xq: torch.Tensor            # [T_tot, H, d]
+    xk: torch.Tensor            # [T_tot, H, d]
+    xv: torch.Tensor            # [T_tot, H, d]
+    wq: torch.Tensor            # [H, d, 4] fp32 filter taps
+    wk: torch.Tensor
+    wv: torch.Tensor
+    beta_raw: torch.Tensor      # [T_tot, H]
+    g: torch.Tensor             # [T_tot, H, d] raw gate
+    z: torch.Tensor             # [T_tot, H, d] raw output-gate projection
+    cu_seqlens: torch.Tensor    # [N+1] int32
+
+
+def make_layer(lengths, H: int, d: int, dtype=torch.bfloat16, seed: int = 0,
+               w_std: float = 0.5, device=None) -> LayerInputs:
+    """Raw projections x ~ N(0, 1), filter taps ~ N(0, w_std^2) (fp32),
+    beta_raw, g, z ~ N(0, 1); drawn in fp32, rounded to dtype (taps stay fp32)."""
+    dev = torch.device("cpu") if device is None else torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(int(seed))
+    T = int(sum(lengths))
+    kw = dict(generator=gen, device=dev)
+    xq, xk, xv = (torch.randn(T, H, d, **kw).to(dtype) for _ in range(3))
+    wq, wk, wv = (torch.randn(H, d, 4, **kw) * float(w_std) for _ in range(3))
+    beta_raw = torch.randn(T, H, **kw).to(dtype)
+    g = torch.randn(T, H, d, **kw).to(dtype)
+    z = torch.randn(T, H, d, **kw).to(dtype)
+    return LayerInputs(xq, xk, xv, wq, wk, wv, beta_raw, g, z, cu_from_lengths(lengths).to(dev))

@@ -114,6 +114,29 @@ KDA_API kda_status kda_chunk_fwd(const void *q, const void *k, const void *v,
                          size_t workspace_bytes, void *stream);
 
 /*
+ * kda_chunk_fwd with the output gate fused into the output store:
+ *
+ *   o_t = (S_t^T q_t) * sigmoid(z_t)     elementwise over the dv channels
+ *
+ * Page "Kimi K3 发布核实与 Moonshot AI 主干架构演变", §3 "K3 对 Kimi Linear 的
+ * 进一步修改", bullet 2: the output gate is an input-dependent, full-rank
+ * channel gate; reading: o * sigmoid(z) per value channel, no normalisation.
+ *
+ *   z   device [T_tot, H, dv] (dt), the raw gate projection; required when
+ *       T_tot > 0 (KDA_ERR_INVALID_ARGUMENT otherwise), 16-byte aligned.
+ *
+ * Every other argument, the workspace and the status contract are those of
+ * kda_chunk_fwd; hT is the ungated final state.  The gate is applied to the
+ * fp32 output values in registers, before the single rounding to dt.
+ */
+KDA_API kda_status kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
+                                       const void *g, const void *beta, const float *h0,
+                                       const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                                       int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                       const void *z, void *o, float *hT, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/*
  * One decode step for B sequences x H heads: one token each.  Same
  * recurrence as the prefill (one token of it); S is updated in place.
  *
@@ -131,6 +154,41 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const void *g, const void *beta, float *S,
                            void *o, int32_t B, int32_t H, int32_t dk,
                            int32_t dv, kda_dtype dt, void *stream);
+
+/*
+ * The step just before the operator, fused into one memory-bound pass: the
+ * operator's inputs q, k, v, beta from the raw projections of the layer.
+ * Page "Kimi K3 模型架构解析：KDA、AttnRes 与 Stable LatentMoE", §二.3 (a
+ * length-4 short convolution mixes neighbouring tokens); readings where the
+ * page is silent: the convolution is causal and depthwise, it restarts at
+ * every sequence start, no activation follows it, and q and k are then
+ * L2-normalised per (token, head):
+ *
+ *   q_t = xq'_t / |xq'_t|,  k_t = xk'_t / |xk'_t|,  v_t = xv'_t,
+ *   x'_t = sum_{j=0..3} w[:, :, j] * x_{t-j}   (tokens before the sequence
+ *                                               start count as zero)
+ *   beta_t = sigmoid(beta_raw_t)
+ *
+ * An all-zero convolved row of q or k stays zero.  The gate g is not touched
+ * (kda_chunk_fwd applies log a = -5 sigmoid(g) itself).
+ *
+ *   xq, xk, xv  device [T_tot, H, d]  (dt)  raw projections
+ *   wq, wk, wv  device [H, d, 4] fp32       filter taps (tap j: token t - j)
+ *   beta_raw    device [T_tot, H]     (dt)
+ *   cu_seqlens  as for kda_chunk_fwd (NULL: N sequences of T_tot / N)
+ *   q, k, v     device [T_tot, H, d]  (dt)  outputs (may not alias the inputs)
+ *   beta        device [T_tot, H]     (dt)  output
+ *
+ * d in {16, 32, 64, 128}; dt KDA_BF16 or KDA_FP32 (fp32 arithmetic, outputs
+ * rounded to dt); H <= 65535.  Argument errors are reported before any
+ * launch; a malformed cu_seqlens is reported by kda_stream_status() as
+ * KDA_ERR_BAD_SEQLENS (every access stays inside the buffers).
+ */
+KDA_API kda_status kda_prologue(const void *xq, const void *xk, const void *xv,
+                                const float *wq, const float *wk, const float *wv,
+                                const void *beta_raw, const int32_t *cu_seqlens, int32_t N,
+                                int64_t T_tot, int32_t H, int32_t d, kda_dtype dt, void *q,
+                                void *k, void *v, void *beta, void *stream);
 
 /*
  * kda_chunk_fwd without a caller-provided workspace, for callers that cannot

@@ -177,3 +177,26 @@ def test_prefill_stall_diagnostic_checks_its_arguments(lib):
     assert lib.kda_debug_stall_prefill(-1, 1000) == binding.KDA_ERR_INVALID_ARGUMENT
     assert lib.kda_debug_stall_prefill(0, 0) == binding.KDA_ERR_INVALID_ARGUMENT
     assert lib.kda_debug_stall_prefill(0, (1 << 32) + 1) == binding.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_prologue_arguments_checked_on_the_host(lib):
+    """Unsupported head sizes and dtypes, bad counts and NULL pointers are
+    refused before any launch (the pointers below are never dereferenced)."""
+    P = ctypes.c_void_p
+    args = lambda d, H, N, T, dt, x=P(256): (x, P(256), P(256), P(256), P(256), P(256), P(256),
+                                             None, N, T, H, d, dt, P(256), P(256), P(256),
+                                             P(256), None)
+    assert lib.kda_prologue(*args(48, 2, 1, 64, binding.KDA_BF16)) == binding.KDA_ERR_UNSUPPORTED
+    assert lib.kda_prologue(*args(128, 2, 1, 64, 7)) == binding.KDA_ERR_UNSUPPORTED
+    assert lib.kda_prologue(*args(128, 0, 1, 64, binding.KDA_BF16)) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_prologue(*args(128, 70000, 1, 64, binding.KDA_BF16)) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_prologue(*args(128, 2, 3, 64, binding.KDA_BF16)) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_prologue(*args(128, 2, 1, 64, binding.KDA_BF16, None)) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_prologue(*args(128, 2, 0, 0, binding.KDA_BF16)) == binding.KDA_OK
+
+
+def test_gated_prefill_needs_z(lib):
+    P = ctypes.c_void_p
+    st = lib.kda_chunk_fwd_gated(P(256), P(256), P(256), P(256), P(256), None, None, 1, 64, 2,
+                                 128, 128, binding.KDA_BF16, None, P(256), None, None, 0, None)
+    assert st == binding.KDA_ERR_INVALID_ARGUMENT
