@@ -74,6 +74,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_version.argtypes = []
     lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.kda_chunk_fwd_softplus.restype = ctypes.c_int
+    lib.kda_chunk_fwd_softplus.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                           i32, ctypes.c_int, vp, vp, vp]
+    lib.kda_decode_step_softplus.restype = ctypes.c_int
+    lib.kda_decode_step_softplus.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                             i32, ctypes.c_int, vp]
     lib.kda_prologue.restype = ctypes.c_int
     lib.kda_prologue.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                  ctypes.c_int, vp, vp, vp, vp, vp]
@@ -266,7 +272,7 @@ def kda_chunk_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     g: torch.Tensor, beta: torch.Tensor, S: torch.Tensor, *,
                     o: Optional[torch.Tensor] = None,
-                    stream=None) -> torch.Tensor:
+                    stream=None, _softplus: bool = False) -> torch.Tensor:
     """One KDA decode step; S [B,H,dk,dv] fp32 is updated in place.
     Returns o [B, H, dv] (dtype of q)."""
     lib = load_library()
@@ -284,12 +290,61 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if o is None:
         o = torch.empty(B, H, dv, dtype=dt, device=dev)
     _check(o, "o", dt, (B, H, dv), dev)
-    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                             _ptr(S), _ptr(o), B, H, dk, dv, _DTYPES[dt],
-                             _stream_handle(stream))
+    fn = lib.kda_decode_step_softplus if _softplus else lib.kda_decode_step
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), B, H, dk, dv,
+            _DTYPES[dt], _stream_handle(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_decode_step")
+        raise KdaError(st, "kda_decode_step" + ("_softplus" if _softplus else ""))
     return o
+
+
+def kda_decode_step_softplus(q, k, v, g, beta, S, *, o=None, stream=None) -> torch.Tensor:
+    """kda_decode_step with the unbounded gate log a = -softplus(g)."""
+    return kda_decode_step(q, k, v, g, beta, S, o=o, stream=stream, _softplus=True)
+
+
+def kda_chunk_fwd_softplus(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           g: torch.Tensor, beta: torch.Tensor,
+                           h0: Optional[torch.Tensor] = None,
+                           cu_seqlens: Optional[torch.Tensor] = None, *,
+                           num_seqs: Optional[int] = None,
+                           o: Optional[torch.Tensor] = None,
+                           hT: Optional[torch.Tensor] = None,
+                           output_final_state: bool = True,
+                           stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked prefill with the unbounded gate log a = -softplus(g) (fp32
+    CUDA-core path, any supported head size, bf16 or fp32 inputs)."""
+    lib = load_library()
+    dev = q.device
+    T_tot, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name, shp in ((q, "q", (T_tot, H, dk)), (k, "k", (T_tot, H, dk)),
+                         (g, "g", (T_tot, H, dk)), (v, "v", (T_tot, H, dv)),
+                         (beta, "beta", (T_tot, H))):
+        _check(t, name, dt, shp, dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty(T_tot, H, dv, dtype=dt, device=dev)
+    _check(o, "o", dt, (T_tot, H, dv), dev)
+    if hT is None and output_final_state:
+        hT = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    st = lib.kda_chunk_fwd_softplus(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                    _ptr(h0), _ptr(cu_seqlens), N, T_tot, H, dk, dv,
+                                    _DTYPES[dt], _ptr(o), _ptr(hT), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_softplus")
+    return o, hT
 
 
 def kda_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:

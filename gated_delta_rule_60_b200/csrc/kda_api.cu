@@ -29,13 +29,13 @@ inline bool supported_simt_d(int d) {
     return d == 16 || d == 32 || d == 64 || d == 128;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kSoftplus = false>
 kda_status launch_simt(const void *q, const void *k, const void *v,
                        const void *g, const void *beta, const float *h0,
                        const int32_t *cu, int N, int64_t T_tot, int H,
                        const void *z, void *o, float *hT, cudaStream_t s) {
     const size_t smem = sizeof(kda::SimtSmem<D>);
-    auto kern = kda::chunk_fwd_simt_kernel<T, D>;
+    auto kern = kda::chunk_fwd_simt_kernel<T, D, kSoftplus>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return KDA_ERR_CUDA;
@@ -45,16 +45,16 @@ kda_status launch_simt(const void *q, const void *k, const void *v,
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-template <typename T>
+template <typename T, bool kSoftplus = false>
 kda_status dispatch_simt(int d, const void *q, const void *k, const void *v,
                          const void *g, const void *beta, const float *h0,
                          const int32_t *cu, int N, int64_t T_tot, int H,
                          const void *z, void *o, float *hT, cudaStream_t s) {
     switch (d) {
-    case 16: return launch_simt<T, 16>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
-    case 32: return launch_simt<T, 32>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
-    case 64: return launch_simt<T, 64>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
-    case 128: return launch_simt<T, 128>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 16: return launch_simt<T, 16, kSoftplus>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 32: return launch_simt<T, 32, kSoftplus>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 64: return launch_simt<T, 64, kSoftplus>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
+    case 128: return launch_simt<T, 128, kSoftplus>(q, k, v, g, beta, h0, cu, N, T_tot, H, z, o, hT, s);
     default: return KDA_ERR_UNSUPPORTED;
     }
 }
@@ -87,28 +87,28 @@ kda_status dispatch_prologue(int d, const void *xq, const void *xk, const void *
     }
 }
 
-template <typename T, int D, int SPLIT>
+template <typename T, int D, int SPLIT, bool kSoftplus = false>
 kda_status launch_decode(const void *q, const void *k, const void *v,
                          const void *g, const void *beta, float *S, void *o,
                          long units, cudaStream_t s) {
     using Sh = kda::DecodeShape<D, SPLIT>;
     const long blocks = (units + Sh::kHeadsPerBlock - 1) / Sh::kHeadsPerBlock;
-    kda::decode_step_kernel<T, D, SPLIT><<<(unsigned)blocks, Sh::kThreads, 0, s>>>(
+    kda::decode_step_kernel<T, D, SPLIT, kSoftplus><<<(unsigned)blocks, Sh::kThreads, 0, s>>>(
         (const T *)q, (const T *)k, (const T *)v, (const T *)g,
         (const T *)beta, S, (T *)o, units);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-template <typename T>
+template <typename T, bool kSoftplus = false>
 kda_status dispatch_decode(int d, const void *q, const void *k, const void *v,
                            const void *g, const void *beta, float *S, void *o,
                            long units, cudaStream_t s) {
     switch (d) {
-    case 16: return launch_decode<T, 16, 1>(q, k, v, g, beta, S, o, units, s);
-    case 32: return launch_decode<T, 32, 1>(q, k, v, g, beta, S, o, units, s);
-    case 64: return launch_decode<T, 64, 1>(q, k, v, g, beta, S, o, units, s);
+    case 16: return launch_decode<T, 16, 1, kSoftplus>(q, k, v, g, beta, S, o, units, s);
+    case 32: return launch_decode<T, 32, 1, kSoftplus>(q, k, v, g, beta, S, o, units, s);
+    case 64: return launch_decode<T, 64, 1, kSoftplus>(q, k, v, g, beta, S, o, units, s);
     case 128:
-        kda::decode_step_d128_kernel<T><<<(unsigned)units, kda::kDecode128Threads, 0, s>>>(
+        kda::decode_step_d128_kernel<T, kSoftplus><<<(unsigned)units, kda::kDecode128Threads, 0, s>>>(
             (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta, S, (T *)o);
         return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     default: return KDA_ERR_UNSUPPORTED;
@@ -204,10 +204,37 @@ kda_status kda_chunk_fwd_gated(const void *q, const void *k, const void *v,
                           workspace, workspace_bytes, stream);
 }
 
-kda_status kda_decode_step(const void *q, const void *k, const void *v,
-                           const void *g, const void *beta, float *S, void *o,
-                           int32_t B, int32_t H, int32_t dk, int32_t dv,
-                           kda_dtype dt, void *stream) {
+kda_status kda_chunk_fwd_softplus(const void *q, const void *k, const void *v,
+                                  const void *g, const void *beta, const float *h0,
+                                  const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                                  int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                  void *o, float *hT, void *stream) {
+    if (N < 0 || T_tot < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
+    if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
+    if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return T_tot == 0 ? KDA_OK : KDA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens == nullptr && (T_tot % N) != 0) return KDA_ERR_INVALID_ARGUMENT;
+    if ((int64_t)N * H > 0x7fffffff) return KDA_ERR_INVALID_ARGUMENT;
+    if (T_tot > 0) {
+        const void *req[] = {q, k, v, g, beta, o};
+        for (const void *p : req)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if ((h0 && !aligned16(h0)) || (hT && !aligned16(hT)) ||
+        (cu_seqlens && !aligned16(cu_seqlens)))
+        return KDA_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == KDA_BF16)
+        return dispatch_simt<__nv_bfloat16, true>(dk, q, k, v, g, beta, h0, cu_seqlens, N, T_tot,
+                                                  H, nullptr, o, hT, s);
+    return dispatch_simt<float, true>(dk, q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H,
+                                      nullptr, o, hT, s);
+}
+
+static kda_status decode_impl(const void *q, const void *k, const void *v, const void *g,
+                              const void *beta, float *S, void *o, int32_t B, int32_t H,
+                              int32_t dk, int32_t dv, kda_dtype dt, bool softplus,
+                              void *stream) {
     if (B < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
     if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
     if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
@@ -218,9 +245,27 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
         if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const long units = (long)B * H;
+    if (softplus)
+        return dt == KDA_BF16
+                   ? dispatch_decode<__nv_bfloat16, true>(dk, q, k, v, g, beta, S, o, units, s)
+                   : dispatch_decode<float, true>(dk, q, k, v, g, beta, S, o, units, s);
     if (dt == KDA_BF16)
         return dispatch_decode<__nv_bfloat16>(dk, q, k, v, g, beta, S, o, units, s);
     return dispatch_decode<float>(dk, q, k, v, g, beta, S, o, units, s);
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *g, const void *beta, float *S, void *o,
+                           int32_t B, int32_t H, int32_t dk, int32_t dv,
+                           kda_dtype dt, void *stream) {
+    return decode_impl(q, k, v, g, beta, S, o, B, H, dk, dv, dt, false, stream);
+}
+
+kda_status kda_decode_step_softplus(const void *q, const void *k, const void *v,
+                                    const void *g, const void *beta, float *S, void *o,
+                                    int32_t B, int32_t H, int32_t dk, int32_t dv,
+                                    kda_dtype dt, void *stream) {
+    return decode_impl(q, k, v, g, beta, S, o, B, H, dk, dv, dt, true, stream);
 }
 
 kda_status kda_prologue(const void *xq, const void *xk, const void *xv, const float *wq,

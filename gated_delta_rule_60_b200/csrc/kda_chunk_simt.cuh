@@ -18,6 +18,14 @@
 // Rows past the end of a sequence are padded with exact no-op tokens
 // (k = q = v = 0, beta = 0, log-decay 0).
 //
+// kSoftplus: the unbounded gate log a = -softplus(g).  A chunk's cumulative
+// log-decay is then unbounded, so the centred split e^{b-m} e^{m-b} can leave
+// the fp32 range; every decay factor is formed instead as the exponential of
+// a direct sum over the tokens it spans (prefix sums from the chunk start,
+// suffix sums from its end, and for A and M the sum over tokens i+1 .. r of
+// each pair), all <= 0, so each factor lies in [0, 1] and a token that forgets
+// everything (g = +inf) gives exact zeros rather than -inf - (-inf).
+//
 // One CTA runs one (sequence, head) chain over all of its chunks; the state
 // lives in shared memory in fp32.  With z given, every output row is
 // multiplied by sigmoid(z) before it is stored (the fused output gate).
@@ -41,7 +49,7 @@ struct SimtSmem {
     float beta[kChunk];
 };
 
-template <typename T, int D>
+template <typename T, int D, bool kSoftplus = false>
 __global__ void __launch_bounds__(256)
 chunk_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, const T *__restrict__ g,
@@ -71,7 +79,7 @@ chunk_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                 qv = IO<T>::ld(q + x);
                 kv = IO<T>::ld(k + x);
                 vv = IO<T>::ld(v + x);
-                lv = log_decay(IO<T>::ld(g + x));
+                lv = kSoftplus ? log_decay_softplus(IO<T>::ld(g + x)) : log_decay(IO<T>::ld(g + x));
             }
             sm.q[r][c] = qv; sm.k[r][c] = kv; sm.v[r][c] = vv; sm.l[r][c] = lv;
         }
@@ -79,7 +87,25 @@ chunk_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
             sm.beta[tid] = tid < L ? IO<T>::ld(beta + (size_t)(c0 + tid) * H + h) : 0.f;
         __syncthreads();
         // 2. per channel: cumulative log-decay and the scaled operands
-        for (int c = tid; c < D; c += 256) {
+        for (int c = tid; c < D && kSoftplus; c += 256) {
+            // prefix sums b_r from the chunk start, suffix sums from its end
+            float b[kChunk], sfx[kChunk];
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < kChunk; ++r) { acc += sm.l[r][c]; b[r] = acc; }
+            acc = 0.f;
+#pragma unroll
+            for (int r = kChunk - 1; r >= 0; --r) { sfx[r] = acc; acc += sm.l[r][c]; }
+            sm.gam[c] = expf(b[kChunk - 1]);
+#pragma unroll
+            for (int r = 0; r < kChunk; ++r) {
+                const float kr = sm.k[r][c], qr = sm.q[r][c];
+                sm.Qa[r][c] = qr * expf(b[r]);
+                sm.Ka[r][c] = kr * expf(b[r]);
+                sm.Ke[r][c] = kr * expf(sfx[r]);
+            }
+        }
+        for (int c = tid; c < D && !kSoftplus; c += 256) {
             float b[kChunk];
             float acc = 0.f;
 #pragma unroll
@@ -102,9 +128,21 @@ chunk_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
         {
             const int r = tid / kChunk, i = tid % kChunk;
             float akk = 0.f, aqk = 0.f;
-            for (int c = 0; c < D; ++c) {
-                akk = fmaf(sm.Kr[r][c], sm.Kh[i][c], akk);
-                aqk = fmaf(sm.Qr[r][c], sm.Kh[i][c], aqk);
+            if (kSoftplus) {
+                // decay between token i and token r: e^{l_{i+1} + .. + l_r}
+                if (i <= r)
+                    for (int c = 0; c < D; ++c) {
+                        float sp = 0.f;
+                        for (int t = i + 1; t <= r; ++t) sp += sm.l[t][c];
+                        const float w = expf(sp) * sm.k[i][c];
+                        akk = fmaf(sm.k[r][c], w, akk);
+                        aqk = fmaf(sm.q[r][c], w, aqk);
+                    }
+            } else {
+                for (int c = 0; c < D; ++c) {
+                    akk = fmaf(sm.Kr[r][c], sm.Kh[i][c], akk);
+                    aqk = fmaf(sm.Qr[r][c], sm.Kh[i][c], aqk);
+                }
             }
             sm.A[r][i] = i < r ? sm.beta[r] * akk : 0.f;
             sm.M[r][i] = i <= r ? aqk : 0.f;

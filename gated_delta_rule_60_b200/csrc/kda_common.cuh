@@ -46,6 +46,13 @@ __device__ __forceinline__ float out_gate(float z) {
     return 1.0f / (1.0f + __expf(-z));
 }
 
+// The unbounded gate of Kimi Linear that K3 replaced (same page, same bullet):
+// log a = -softplus(g), in fp32, stable for every g (g = +inf gives -inf,
+// g = -inf gives 0).
+__device__ __forceinline__ float log_decay_softplus(float g) {
+    return -(fmaxf(g, 0.f) + log1pf(expf(-fabsf(g))));
+}
+
 template <typename T>
 struct IO;
 

@@ -31,7 +31,8 @@ struct DecodeShape {
     static constexpr int kThreads = kHeadsPerBlock * kThreadsPerHead;
 };
 
-template <typename T, int D, int SPLIT>
+// kSoftplus: the unbounded gate log a = -softplus(g) instead of -5 sigmoid(g).
+template <typename T, int D, int SPLIT, bool kSoftplus = false>
 __global__ void __launch_bounds__(DecodeShape<D, SPLIT>::kThreads)
 decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
                    const T *__restrict__ v, const T *__restrict__ g,
@@ -58,7 +59,8 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
             const size_t e = (size_t)u * D + j;
             sq[hl][j] = IO<T>::ld(q + e);
             sk[hl][j] = IO<T>::ld(k + e);
-            sa[hl][j] = expf(log_decay(IO<T>::ld(g + e)));
+            const float gv = IO<T>::ld(g + e);
+            sa[hl][j] = expf(kSoftplus ? log_decay_softplus(gv) : log_decay(gv));
         }
     }
     __syncthreads();
@@ -120,7 +122,7 @@ __device__ __forceinline__ void st_stream_f4(float *p, float4 v) {
 
 constexpr int kDecode128Threads = 256;
 
-template <typename T>
+template <typename T, bool kSoftplus = false>
 __global__ void __launch_bounds__(kDecode128Threads)
 decode_step_d128_kernel(const T *__restrict__ q, const T *__restrict__ k,
                         const T *__restrict__ v, const T *__restrict__ g,
@@ -139,7 +141,8 @@ decode_step_d128_kernel(const T *__restrict__ q, const T *__restrict__ k,
         const size_t e = (size_t)u * D + tid;
         sq[tid] = IO<T>::ld(q + e);
         sk[tid] = IO<T>::ld(k + e);
-        sa[tid] = expf(log_decay(IO<T>::ld(g + e)));
+        const float gv = IO<T>::ld(g + e);
+        sa[tid] = expf(kSoftplus ? log_decay_softplus(gv) : log_decay(gv));
     }
     __syncthreads();
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;

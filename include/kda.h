@@ -156,6 +156,32 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            int32_t dv, kda_dtype dt, void *stream);
 
 /*
+ * The operator with the unbounded gate of Kimi Linear, the one K3 replaced
+ * (page "Kimi K3 发布核实与 Moonshot AI 主干架构演变", §3 "K3 对 Kimi Linear
+ * 的进一步修改", bullet 1):
+ *
+ *   log a_t = -softplus(g_t)            (instead of -5 sigmoid(g_t))
+ *
+ * Without the -5 bound a 16-token tile's cumulative decay can leave the BF16
+ * and fp32 ranges, so this variant runs on the fp32 CUDA-core chunk kernel
+ * with every decay factor formed as the exponential of a direct sum over the
+ * tokens it spans (each factor in [0, 1]; g = +inf forgets exactly).
+ * Arguments, layouts and status as for kda_chunk_fwd (no workspace); dt
+ * KDA_BF16 or KDA_FP32, dk = dv in {16, 32, 64, 128}.
+ */
+KDA_API kda_status kda_chunk_fwd_softplus(const void *q, const void *k, const void *v,
+                                          const void *g, const void *beta, const float *h0,
+                                          const int32_t *cu_seqlens, int32_t N, int64_t T_tot,
+                                          int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                                          void *o, float *hT, void *stream);
+
+/* kda_decode_step with the unbounded gate log a = -softplus(g) (see above). */
+KDA_API kda_status kda_decode_step_softplus(const void *q, const void *k, const void *v,
+                                            const void *g, const void *beta, float *S,
+                                            void *o, int32_t B, int32_t H, int32_t dk,
+                                            int32_t dv, kda_dtype dt, void *stream);
+
+/*
  * The step just before the operator, fused into one memory-bound pass: the
  * operator's inputs q, k, v, beta from the raw projections of the layer.
  * Page "Kimi K3 模型架构解析：KDA、AttnRes 与 Stable LatentMoE", §二.3 (a
