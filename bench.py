@@ -44,25 +44,56 @@ FLOPS_PER_TOKEN_HEAD = 2 * 128 * 128 * 3 + 2 * 16 * 128 * 5   # 118,784
 STATE_BYTES = 128 * 128 * 4
 
 
-def _measured_traffic():
-    """DRAM bytes per launch of the prefill kernel from the committed ncu
-    summary, or None when the kernel sources changed since that capture."""
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "chunk_fwd_sm100_k3_prefill.json")
+PREFILL_SOURCES = ("kda_chunk_sm100.cuh", "sm100_ptx.cuh", "kda_common.cuh")
+
+
+def _prefill_source_hash():
     import hashlib
-    srcs = [os.path.join(ROOT, "gated_delta_rule_60_b200", "csrc", f)
-            for f in ("kda_chunk_sm100.cuh", "sm100_ptx.cuh")]
+    srcs = [os.path.join(ROOT, "gated_delta_rule_60_b200", "csrc", f) for f in PREFILL_SOURCES]
+    return hashlib.sha256(b"".join(open(f, "rb").read() for f in srcs)).hexdigest()[:16]
+
+
+def _measured_traffic():
+    """DRAM bytes (read + write) per launch of the prefill kernel, from the
+    committed ncu record, or None when the kernel sources changed since that
+    capture."""
     try:
-        h = hashlib.sha256(b"".join(open(f, "rb").read() for f in srcs)).hexdigest()[:16]
-        text = open(os.path.join(ROOT, "profiles", "chunk_fwd_sm100_k3_prefill.md")).read()
-    except OSError:
+        rec = json.load(open(TRAFFIC_JSON))
+        if rec.get("kernel_source_sha256_16") != _prefill_source_hash():
+            return None
+        return float(rec["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
         return None
-    fields = dict(line.split(":", 1) for line in text.splitlines()
-                  if line.startswith(("kernel-source-sha256-16:", "traffic_bytes_per_launch:")))
-    if fields.get("kernel-source-sha256-16", "").strip() != h:
-        return None
-    val = fields.get("traffic_bytes_per_launch", "").strip().split()
-    if len(val) != 2 or val[1] != "kB":
-        return None
-    return float(val[0]) * 1e3
+
+
+def record_traffic(csv_path, command):
+    """Write the ncu DRAM counters of one prefill launch (an ncu --csv log of
+    dram__bytes_read.sum and dram__bytes_write.sum) to the traffic record,
+    keyed by the current kernel source hash."""
+    import csv
+    vals = {}
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(f) if len(r) > 5]
+    hdr = rows[0]
+    for r in rows[1:]:
+        d = dict(zip(hdr, r))
+        if "chunk_fwd_sm100" not in d.get("Kernel Name", ""):
+            continue
+        name, unit = d["Metric Name"], d.get("Metric Unit", "")
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit)
+        if scale is None:
+            raise ValueError("unexpected unit %r for %s" % (unit, name))
+        vals[name] = float(d["Metric Value"].replace(",", "")) * scale
+    rd, wr = vals["dram__bytes_read.sum"], vals["dram__bytes_write.sum"]
+    rec = {"kernel": "chunk_fwd_sm100_kernel (K3 prefill: B=1 H=96 T=8192 d=128 bf16)",
+           "kernel_source_sha256_16": _prefill_source_hash(),
+           "dram_bytes_read": rd, "dram_bytes_write": wr,
+           "traffic_bytes_per_launch": rd + wr, "command": command}
+    with open(TRAFFIC_JSON, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    print(json.dumps(rec))
 
 
 def _peaks():
@@ -380,34 +411,64 @@ def _measure_workload(w, dev, stream, args, world, hbm_peak, binding, inputs):
 
 
 def _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding):
-    host = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
-    o_host = torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory()
-    h_host = torch.empty(1, H, d, d, dtype=torch.float32).pin_memory()
+    """End to end through the public API: every step copies its inputs from
+    pinned host memory, runs kda_chunk_fwd and reads o and hT back.  Steps are
+    pipelined over two buffer sets: the host-to-device copy of step i+1 and the
+    device-to-host copy of step i-1 run on their own streams while step i
+    computes (events order each buffer's reuse)."""
+    names = ("q", "k", "v", "g", "beta")
+    host = {n: getattr(inp, n).pin_memory() for n in names}
+    o_host = [torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    h_host = [torch.empty(1, H, d, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+    dev_in = [{n: torch.empty_like(t, device=dev) for n, t in host.items()} for _ in range(2)]
+    dev_o = [o, torch.empty_like(o)]
+    dev_h = [hT, torch.empty_like(hT)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_host.numel() * 2 + h_host.numel() * 4
+    d2h = o_host[0].numel() * 2 + h_host[0].numel() * 4
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    n_steps = max(2, min(args.steps, 10))
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev() for _ in range(n_steps + 1)]
+    done = [ev() for _ in range(n_steps + 1)]
+    out_read = [ev() for _ in range(n_steps + 1)]
 
-    def e2e_step():
-        xs = {n: t.to(dev, non_blocking=True) for n, t in host.items()}
-        binding.kda_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"],
-                              None, cu, o=o, hT=hT, workspace=ws, stream=stream)
-        o_host.copy_(o, non_blocking=True)
-        h_host.copy_(hT, non_blocking=True)
+    def run(n, t0=None):
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[i - 2])          # the kernel of step i-2 read buffer b
+                for name in names:
+                    dev_in[b][name].copy_(host[name], non_blocking=True)
+                in_ready[i].record(s_in)
+            stream.wait_event(in_ready[i])
+            if i >= 2:
+                stream.wait_event(out_read[i - 2])        # o, hT of buffer b were read back
+            x = dev_in[b]
+            binding.kda_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, cu,
+                                  o=dev_o[b], hT=dev_h[b], workspace=ws, stream=stream)
+            done[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i])
+                o_host[b].copy_(dev_o[b], non_blocking=True)
+                h_host[b].copy_(dev_h[b], non_blocking=True)
+                out_read[i].record(s_out)
 
-    e2e_steps = max(2, min(args.steps, 10))
-    with torch.cuda.stream(stream):
-        e2e_step()
-        stream.synchronize()
-        _barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-    stream.synchronize()
-    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    run(2)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    run(n_steps)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(stream)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / n_steps, world)
     e2e_val = world * T / (e2e_ms * 1e-3) / 1e6
+    del dev_in
     return {"value": e2e_val, "unit": "Mtok/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h, "pipelined": "2 buffer sets; H2D, compute, D2H on 3 streams"}
 
 
 def _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads):
@@ -526,7 +587,15 @@ def main():
                     help="skip the varlen and long-context prefill measurements")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part only (for profiling): the K3 prefill or the decode")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV", default=None,
+                    help="write the prefill DRAM traffic record from an ncu --csv log of "
+                         "dram__bytes_read.sum and dram__bytes_write.sum (no GPU needed)")
+    ap.add_argument("--record-command", default="",
+                    help="the ncu command line that produced NCU_CSV (kept in the record)")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.record_command)
+        return 0
     if args.impl == "reference":
         return run_reference(args)
     rc = run_gpu(args)

@@ -104,3 +104,30 @@ def test_default_run_on_cpu_fails_loudly():
     r = _run_bench(["--steps", "1", "--warmup", "3"], {"WORLD_SIZE": "1"}, timeout=300)
     assert r.returncode != 0
     assert not any(ln.startswith("{") for ln in r.stdout.splitlines())
+
+
+def test_traffic_record_round_trip(tmp_path, monkeypatch):
+    """bench.py --record-traffic reads an ncu CSV log, keeps the prefill
+    kernel's DRAM counters (converting the units), keys them by the kernel
+    source hash, and the roofline reads them back only while that hash holds."""
+    import bench
+    csv_text = (
+        '"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream",'
+        '"Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit",'
+        '"Metric Value"\n'
+        '"0","1","python","h","void kda::decode_step_kernel","1","7","(256,1,1)","(9,1,1)","0",'
+        '"10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","5.00"\n'
+        '"1","1","python","h","prefill::chunk_fwd_sm100_kernel<false>(...)","1","7","(512,1,1)",'
+        '"(96,1,1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte",'
+        '"809.60"\n'
+        '"1","1","python","h","prefill::chunk_fwd_sm100_kernel<false>(...)","1","7","(512,1,1)",'
+        '"(96,1,1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Kbyte",'
+        '"186,400.00"\n')
+    log = tmp_path / "k3.csv"
+    log.write_text(csv_text)
+    rec_path = tmp_path / "rec.json"
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(rec_path))
+    bench.record_traffic(str(log), "ncu ... (test)")
+    assert bench._measured_traffic() == pytest.approx(809.6e6 + 186.4e6)
+    monkeypatch.setattr(bench, "_prefill_source_hash", lambda: "0" * 16)
+    assert bench._measured_traffic() is None
