@@ -81,6 +81,8 @@ def record_traffic(csv_path, command):
         if "chunk_fwd_sm100" not in d.get("Kernel Name", ""):
             continue
         name, unit = d["Metric Name"], d.get("Metric Unit", "")
+        if not name.startswith("dram__bytes_"):
+            continue
         scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}.get(unit)
         if scale is None:
             raise ValueError("unexpected unit %r for %s" % (unit, name))
