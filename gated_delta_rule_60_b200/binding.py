@@ -74,6 +74,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.kda_version.argtypes = []
     lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.kda_chunk_bwd_workspace_size.restype = sz
+    lib.kda_chunk_bwd_workspace_size.argtypes = [i32, i64, i32, i32, i32, ctypes.c_int]
+    lib.kda_chunk_bwd.restype = ctypes.c_int
+    lib.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                  ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.kda_chunk_fwd_softplus.restype = ctypes.c_int
     lib.kda_chunk_fwd_softplus.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                            i32, ctypes.c_int, vp, vp, vp]
@@ -301,6 +306,50 @@ def kda_decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def kda_decode_step_softplus(q, k, v, g, beta, S, *, o=None, stream=None) -> torch.Tensor:
     """kda_decode_step with the unbounded gate log a = -softplus(g)."""
     return kda_decode_step(q, k, v, g, beta, S, o=o, stream=stream, _softplus=True)
+
+
+def kda_chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, dO: torch.Tensor, h0: Optional[torch.Tensor] = None,
+                  cu_seqlens: Optional[torch.Tensor] = None, dhT: Optional[torch.Tensor] = None,
+                  *, num_seqs: Optional[int] = None, stream=None) -> dict:
+    """Gradient of the prefill for L = <dO, O> + <dhT, hT>: returns a dict of
+    dq, dk, dg [T_tot, H, dk], dv [T_tot, H, dv], dbeta [T_tot, H] (dtype of
+    q) and dh0 [N, H, dk, dv] fp32."""
+    lib = load_library()
+    dev = q.device
+    T_tot, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise TypeError("unsupported dtype %s" % dt)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32, (cu_seqlens.numel(),), dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = 1 if num_seqs is None else int(num_seqs)
+    for t, name, shp in ((q, "q", (T_tot, H, dk)), (k, "k", (T_tot, H, dk)),
+                         (g, "g", (T_tot, H, dk)), (v, "v", (T_tot, H, dv)),
+                         (beta, "beta", (T_tot, H)), (dO, "dO", (T_tot, H, dv))):
+        _check(t, name, dt, shp, dev)
+    for t, name in ((h0, "h0"), (dhT, "dhT")):
+        if t is not None:
+            _check(t, name, torch.float32, (N, H, dk, dv), dev)
+    out = {"dq": torch.empty(T_tot, H, dk, dtype=dt, device=dev),
+           "dk": torch.empty(T_tot, H, dk, dtype=dt, device=dev),
+           "dv": torch.empty(T_tot, H, dv, dtype=dt, device=dev),
+           "dg": torch.empty(T_tot, H, dk, dtype=dt, device=dev),
+           "dbeta": torch.empty(T_tot, H, dtype=dt, device=dev),
+           "dh0": torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)}
+    ws_n = int(lib.kda_chunk_bwd_workspace_size(N, T_tot, H, dk, dv, _DTYPES[dt]))
+    ws = torch.empty(max(ws_n, 256), dtype=torch.uint8, device=dev)
+    st = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                           _ptr(cu_seqlens), N, T_tot, H, dk, dv, _DTYPES[dt], _ptr(dO),
+                           _ptr(dhT), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                           _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dh0"]), _ptr(ws),
+                           ws.numel(), _stream_handle(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_bwd")
+    return out
 
 
 def kda_chunk_fwd_softplus(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -10,6 +10,7 @@
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_sm100.cuh"
 #include "kda_prologue.cuh"
+#include "kda_backward.cuh"
 
 #include <cuda_runtime.h>
 
@@ -83,6 +84,40 @@ kda_status dispatch_prologue(int d, const void *xq, const void *xk, const void *
     case 32: return launch_prologue<T, 32>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
     case 64: return launch_prologue<T, 64>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
     case 128: return launch_prologue<T, 128>(xq, xk, xv, wq, wk, wv, braw, cu, N, T_tot, H, q, k, v, beta, s);
+    default: return KDA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int D>
+kda_status launch_bwd(const void *q, const void *k, const void *v, const void *g,
+                      const void *beta, const float *h0, const int32_t *cu, int N, int64_t T_tot,
+                      int H, const void *dO, const float *dhT, void *dq, void *dk, void *dv,
+                      void *dg, void *dbeta, float *dh0, void *ws, cudaStream_t s) {
+    const size_t smem = sizeof(kda::bwd::Smem<D>);
+    auto kern = kda::bwd::chunk_bwd_kernel<T, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return KDA_ERR_CUDA;
+    const size_t DD = (size_t)D * D;
+    float *ckpt = static_cast<float *>(ws);
+    float *tok = ckpt + (size_t)H * ((T_tot + kda::bwd::kChunk - 1) / kda::bwd::kChunk + N) * DD;
+    kern<<<(unsigned)(N * H), kda::bwd::kThreads, smem, s>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta, h0, cu, N, T_tot,
+        H, (const T *)dO, dhT, (T *)dq, (T *)dk, (T *)dv, (T *)dg, (T *)dbeta, dh0, ckpt, tok);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <typename T>
+kda_status dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *g,
+                        const void *beta, const float *h0, const int32_t *cu, int N,
+                        int64_t T_tot, int H, const void *dO, const float *dhT, void *dq,
+                        void *dk, void *dv, void *dg, void *dbeta, float *dh0, void *ws,
+                        cudaStream_t s) {
+    switch (d) {
+    case 16: return launch_bwd<T, 16>(q, k, v, g, beta, h0, cu, N, T_tot, H, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, s);
+    case 32: return launch_bwd<T, 32>(q, k, v, g, beta, h0, cu, N, T_tot, H, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, s);
+    case 64: return launch_bwd<T, 64>(q, k, v, g, beta, h0, cu, N, T_tot, H, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, s);
+    case 128: return launch_bwd<T, 128>(q, k, v, g, beta, h0, cu, N, T_tot, H, dO, dhT, dq, dk, dv, dg, dbeta, dh0, ws, s);
     default: return KDA_ERR_UNSUPPORTED;
     }
 }
@@ -266,6 +301,47 @@ kda_status kda_decode_step_softplus(const void *q, const void *k, const void *v,
                                     int32_t B, int32_t H, int32_t dk, int32_t dv,
                                     kda_dtype dt, void *stream) {
     return decode_impl(q, k, v, g, beta, S, o, B, H, dk, dv, dt, true, stream);
+}
+
+size_t kda_chunk_bwd_workspace_size(int32_t N, int64_t T_tot, int32_t H, int32_t dk,
+                                    int32_t dv, kda_dtype dt) {
+    if (N <= 0 || T_tot < 0 || H <= 0 || dk != dv || !supported_simt_d(dk)) return 0;
+    if (dt != KDA_BF16 && dt != KDA_FP32) return 0;
+    const size_t DD = (size_t)dk * dk;
+    const size_t ck = (size_t)H * ((size_t)(T_tot + kda::bwd::kChunk - 1) / kda::bwd::kChunk + N);
+    const size_t tok = (size_t)N * H * kda::bwd::kChunk;
+    return (ck + tok) * DD * sizeof(float);
+}
+
+kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
+                         const void *beta, const float *h0, const int32_t *cu_seqlens,
+                         int32_t N, int64_t T_tot, int32_t H, int32_t dk, int32_t dv,
+                         kda_dtype dt, const void *dO, const float *dhT, void *dq, void *dk_,
+                         void *dv_, void *dg, void *dbeta, float *dh0, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    if (N < 0 || T_tot < 0 || H <= 0) return KDA_ERR_INVALID_ARGUMENT;
+    if (dt != KDA_BF16 && dt != KDA_FP32) return KDA_ERR_UNSUPPORTED;
+    if (dk != dv || !supported_simt_d(dk)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0) return T_tot == 0 ? KDA_OK : KDA_ERR_INVALID_ARGUMENT;
+    if (cu_seqlens == nullptr && (T_tot % N) != 0) return KDA_ERR_INVALID_ARGUMENT;
+    if ((int64_t)N * H > 0x7fffffff) return KDA_ERR_INVALID_ARGUMENT;
+    if (T_tot > 0) {
+        const void *req[] = {q, k, v, g, beta, dO, dq, dk_, dv_, dg, dbeta};
+        for (const void *p : req)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if ((h0 && !aligned16(h0)) || (dhT && !aligned16(dhT)) || (dh0 && !aligned16(dh0)) ||
+        (cu_seqlens && !aligned16(cu_seqlens)))
+        return KDA_ERR_INVALID_ARGUMENT;
+    const size_t need = kda_chunk_bwd_workspace_size(N, T_tot, H, dk, dv, dt);
+    if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return KDA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dt == KDA_BF16)
+        return dispatch_bwd<__nv_bfloat16>(dk, q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H, dO,
+                                           dhT, dq, dk_, dv_, dg, dbeta, dh0, workspace, s);
+    return dispatch_bwd<float>(dk, q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H, dO, dhT, dq,
+                               dk_, dv_, dg, dbeta, dh0, workspace, s);
 }
 
 kda_status kda_prologue(const void *xq, const void *xk, const void *xv, const float *wq,

@@ -156,6 +156,41 @@ KDA_API kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            int32_t dv, kda_dtype dt, void *stream);
 
 /*
+ * Gradient of the prefill for L = <dO, O> + <dhT, hT> (training; page "Kimi
+ * K3 发布核实与 Moonshot AI 主干架构演变", §3 "KDA 为什么不同于 MLA", item 3:
+ * the chunked form serves training).  Gate log a = -5 sigmoid(g).
+ *
+ *   q, k, v, g, beta, h0, cu_seqlens, N, T_tot, H, dk, dv, dt  as for
+ *               kda_chunk_fwd (the forward's inputs; the forward's outputs
+ *               are not needed: the state is recomputed)
+ *   dO          device [T_tot, H, dv]  (dt)  gradient of o
+ *   dhT         device [N, H, dk, dv] fp32   gradient of hT, or NULL (= 0)
+ *   dq, dk, dg  device [T_tot, H, dk]  (dt)  outputs
+ *   dv          device [T_tot, H, dv]  (dt)  output
+ *   dbeta       device [T_tot, H]      (dt)  output
+ *   dh0         device [N, H, dk, dv] fp32   output (gradient of the initial
+ *               state, h0 given or not), or NULL (not written)
+ *   workspace   kda_chunk_bwd_workspace_size() bytes, 256-byte aligned:
+ *               the state at every 16-token chunk boundary of every (sequence,
+ *               head), and 16 token states per (sequence, head)
+ *
+ * fp32 arithmetic on CUDA cores: one CTA per (sequence, head) sweeps the
+ * sequence forward keeping chunk-boundary states, then walks the chunks in
+ * reverse, recomputing each chunk's token states from its checkpoint and
+ * applying the token-level chain rule.  dk = dv in {16, 32, 64, 128};
+ * KDA_BF16 or KDA_FP32.  Argument and workspace errors are reported before any
+ * launch; a malformed cu_seqlens is reported by kda_stream_status().
+ */
+KDA_API size_t kda_chunk_bwd_workspace_size(int32_t N, int64_t T_tot, int32_t H, int32_t dk,
+                                            int32_t dv, kda_dtype dt);
+KDA_API kda_status kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
+                                 const void *beta, const float *h0, const int32_t *cu_seqlens,
+                                 int32_t N, int64_t T_tot, int32_t H, int32_t dk, int32_t dv,
+                                 kda_dtype dt, const void *dO, const float *dhT, void *dq,
+                                 void *dk_, void *dv_, void *dg, void *dbeta, float *dh0,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The operator with the unbounded gate of Kimi Linear, the one K3 replaced
  * (page "Kimi K3 发布核实与 Moonshot AI 主干架构演变", §3 "K3 对 Kimi Linear
  * 的进一步修改", bullet 1):

@@ -200,3 +200,16 @@ def test_gated_prefill_needs_z(lib):
     st = lib.kda_chunk_fwd_gated(P(256), P(256), P(256), P(256), P(256), None, None, 1, 64, 2,
                                  128, 128, binding.KDA_BF16, None, P(256), None, None, 0, None)
     assert st == binding.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_backward_workspace_and_arguments(lib):
+    """The backward's workspace grows with the chunk checkpoints; a missing or
+    short workspace is refused before any launch."""
+    ws = lib.kda_chunk_bwd_workspace_size(2, 100, 3, 64, 64, binding.KDA_FP32)
+    assert ws == (3 * ((100 + 15) // 16 + 2) + 2 * 3 * 16) * 64 * 64 * 4
+    assert lib.kda_chunk_bwd_workspace_size(2, 100, 3, 48, 48, binding.KDA_FP32) == 0
+    P = ctypes.c_void_p
+    args = [P(256)] * 5 + [None, None, 1, 64, 2, 64, 64, binding.KDA_FP32, P(256), None] + \
+        [P(256)] * 5 + [None]
+    assert lib.kda_chunk_bwd(*args, None, 0, None) == binding.KDA_ERR_WORKSPACE
+    assert lib.kda_chunk_bwd(*args, P(512), 16, None) == binding.KDA_ERR_WORKSPACE
