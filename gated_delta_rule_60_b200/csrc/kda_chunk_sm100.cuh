@@ -289,15 +289,6 @@ __device__ __forceinline__ float rcp(float x) {
     return y;
 }
 
-// decay factors a = exp(-5 sigmoid(g)) of a channel pair, via exp2
-__device__ __forceinline__ float2 decay2(float2 g) {
-    const float2 x = fmul2(g, make_float2(-kLog2e, -kLog2e));
-    const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), make_float2(1.f, 1.f));
-    const float2 l = fmul2(make_float2(rcp(den.x), rcp(den.y)),
-                           make_float2(-5.f * kLog2e, -5.f * kLog2e));
-    return make_float2(ex2(l.x), ex2(l.y));
-}
-
 // Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort, unsigned long long limit) {
@@ -328,46 +319,50 @@ __host__ __device__ __forceinline__ uint32_t core32_off(uint32_t n, uint32_t k) 
 // Thread (pw, lane) of a prep warpgroup handles rows 16 (pw >> 1) .. + 15
 // and key channels 64 (pw & 1) + 2 lane, + 1.  kFull: all 32 rows are tokens
 // of the sequence (no masking).  Writes eps (first tile) or delta (second).
+// The cumulative log-decay is summed in base 2 (b = sum of -5 log2(e)
+// sigmoid(g)), so each element costs two MUFU operations for the sigmoid
+// and two for e^{b-m} and its reciprocal.
 template <bool kFull>
 __device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane, int Ls,
                                           float *eps_out, float *dlt_out) {
-    const int th = pw >> 1, kb = pw & 1, cc = 2 * lane;
+    const int th = pw >> 1, kb = pw & 1;
     const int r0 = 16 * th;
     const uint32_t oK = kb ? SL_K1 : SL_K0, oQ = kb ? SL_Q1 : SL_Q0;
     const uint32_t oG = kb ? SL_G1 : SL_G0;
+    // element (r0 + rr, 2 lane) of a 128-byte-swizzled box: the 16-byte
+    // chunk (lane >> 2) of row rr moves to chunk (lane >> 2) ^ (rr & 7)
+    const uint32_t cbase = (uint32_t)r0 * 128u + (uint32_t)(lane & 3) * 4u;
+    const uint32_t chunk = (uint32_t)(lane >> 2);
+    const float2 c1 = make_float2(-kLog2e, -kLog2e);
+    const float2 c5 = make_float2(-5.f * kLog2e, -5.f * kLog2e);
     const float2 one = make_float2(1.f, 1.f);
-    float2 eb[kTile];
-    float2 acc = one;
+    float2 bb[kTile];
+    float2 b = make_float2(0.f, 0.f);
 #pragma unroll
     for (int rr = 0; rr < kTile; ++rr) {
-        const int r = r0 + rr;
-        const float2 g = bf16x2_to_float2(
-            *reinterpret_cast<const uint32_t *>(slot + oG + sw128_off(r, cc)));
-        const float2 a = decay2(g);
-        acc = fmul2(acc, (kFull || r < Ls) ? a : one);
-        eb[rr] = acc;
+        const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
+        const float2 g = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(slot + oG + o));
+        const float2 x = fmul2(g, c1);
+        const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), one);
+        const float2 sg = make_float2(rcp(den.x), rcp(den.y));              // sigmoid(g)
+        if (kFull || r0 + rr < Ls) b = ffma2(sg, c5, b);
+        bb[rr] = b;
     }
-    // first tile: b - m = log(eb / eb_15); second tile: b - m = log(eb)
-    const float2 tot = eb[kTile - 1];
-    float2 base = one, top = one;
-    if (th == 0) {
-        base = make_float2(rcp(tot.x), rcp(tot.y));
-        top = tot;
-        *reinterpret_cast<float2 *>(eps_out + 64 * kb + cc) = tot;
-    } else {
-        *reinterpret_cast<float2 *>(dlt_out + 64 * kb + cc) = tot;
-    }
+    const float2 tot = bb[kTile - 1];
+    *reinterpret_cast<float2 *>((th == 0 ? eps_out : dlt_out) + 64 * kb + 2 * lane) =
+        make_float2(ex2(tot.x), ex2(tot.y));
+    // first tile: b - m = b - tot; second tile: b - m = b
+    const float2 nbase = th == 0 ? make_float2(-tot.x, -tot.y) : make_float2(0.f, 0.f);
 #pragma unroll
     for (int rr = 0; rr < kTile; ++rr) {
-        const int r = r0 + rr;
-        const uint32_t o = sw128_off(r, cc);
-        const bool live = kFull || r < Ls;
-        const uint32_t kraw = *reinterpret_cast<const uint32_t *>(slot + oK + o);
-        const uint32_t qraw = *reinterpret_cast<const uint32_t *>(slot + oQ + o);
-        const float2 kf = bf16x2_to_float2(live ? kraw : 0u);
-        const float2 qf = bf16x2_to_float2(live ? qraw : 0u);
-        const float2 er = fmul2(eb[rr], base);                                  // e^{b-m}
-        const float2 ei = fmul2(top, make_float2(rcp(eb[rr].x), rcp(eb[rr].y)));  // e^{m-b}
+        const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
+        const bool live = kFull || r0 + rr < Ls;
+        const float2 dd = fadd2(bb[rr], nbase);
+        const float2 er = make_float2(ex2(dd.x), ex2(dd.y));                // e^{b-m}
+        const float2 ei = make_float2(rcp(er.x), rcp(er.y));                // e^{m-b}
+        const uint32_t kraw = live ? *reinterpret_cast<const uint32_t *>(slot + oK + o) : 0u;
+        const uint32_t qraw = live ? *reinterpret_cast<const uint32_t *>(slot + oQ + o) : 0u;
+        const float2 kf = bf16x2_to_float2(kraw), qf = bf16x2_to_float2(qraw);
         const float2 kr = fmul2(kf, er), qr = fmul2(qf, er), kh = fmul2(kf, ei);
         *reinterpret_cast<uint32_t *>(slot + oK + o) = pack_bf16(kr.x, kr.y);
         *reinterpret_cast<uint32_t *>(slot + oQ + o) = pack_bf16(qr.x, qr.y);
@@ -840,35 +835,92 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             group_sync(bar_id);                                             // scratch written
 
-            // ---------------- T by right-looking forward substitution (solver warp; lane = column)
+            // ---------------- T = M^-1 Diag(beta), M = I + N, N = Diag(beta) strict_lower(A_kk),
+            // by 16 x 16 blocks: M = [M11 0 ; M21 M22], T11 = M11^-1 D1, T22 = M22^-1 D2,
+            // T21 = -M22^-1 (M21 T11).  The scratch at[i][r] = N[r][i] (36-float rows)
+            // also holds the blocks, each where a finished stage no longer reads:
+            //   T11 in at[0..15][0..15], M22^-1 in at[16..31][0..15] (after stage 1),
+            //   Y = M21 T11 in at[16..31][16..31] (stage 2), T21 in at[0..15][16..31] (stage 3).
+            constexpr int kRs = kScRow / 4;
+            float *at = reinterpret_cast<float *>(scr + SC_AT);
+            float tcol[kTile];
+            // (1) solver warp, lane = column: lanes 0-15 invert M11, lanes 16-31 M22
+            //     (right-looking forward substitution inside the block)
             if (pw == solve_w && !*abortp) {
-                const int c = lane;
-                const float bc = bars.beta_s[pg][c];
-                float *at = reinterpret_cast<float *>(scr + SC_AT);
-                float acc[kStep], t[kStep];
+                const int b0 = lane & 16, cc = lane & 15;
+                float acc[kTile];
 #pragma unroll
-                for (int r = 0; r < kStep; ++r) acc[r] = 0.f;
+                for (int r = 0; r < kTile; ++r) acc[r] = 0.f;
 #pragma unroll
-                for (int i = 0; i < kStep; ++i) {
-                    t[i] = (i == c) ? bc : -acc[i];
+                for (int i = 0; i < kTile; ++i) {
+                    tcol[i] = (i == cc ? 1.f : 0.f) - acc[i];
 #pragma unroll
-                    for (int r4 = (i + 1) & ~3; r4 < kStep; r4 += 4) {
-                        const float4 a = *reinterpret_cast<const float4 *>(at + i * (kScRow / 4) + r4);
-                        if (r4 > i) acc[r4] = fmaf(a.x, t[i], acc[r4]);
-                        if (r4 + 1 > i) acc[r4 + 1] = fmaf(a.y, t[i], acc[r4 + 1]);
-                        if (r4 + 2 > i) acc[r4 + 2] = fmaf(a.z, t[i], acc[r4 + 2]);
-                        if (r4 + 3 > i) acc[r4 + 3] = fmaf(a.w, t[i], acc[r4 + 3]);
+                    for (int r4 = (i + 1) & ~3; r4 < kTile; r4 += 4) {
+                        const float4 a = *reinterpret_cast<const float4 *>(at + (b0 + i) * kRs + b0 + r4);
+                        if (r4 > i) acc[r4] = fmaf(a.x, tcol[i], acc[r4]);
+                        if (r4 + 1 > i) acc[r4 + 1] = fmaf(a.y, tcol[i], acc[r4 + 1]);
+                        if (r4 + 2 > i) acc[r4 + 2] = fmaf(a.z, tcol[i], acc[r4 + 2]);
+                        if (r4 + 3 > i) acc[r4 + 3] = fmaf(a.w, tcol[i], acc[r4 + 3]);
                     }
                 }
-                // T bf16: B operand of the Z and P products
+                __syncwarp();
+                // column cc of M_bb^-1: T11 = M11^-1 D1 (lanes 0-15), M22^-1 (lanes 16-31);
+                // tcol becomes the column of T_bb
+                const float bc = bars.beta_s[pg][lane];
 #pragma unroll
-                for (int kg = 0; kg < 4; ++kg) {
+                for (int r = 0; r < kTile; ++r) {
+                    at[(b0 + r) * kRs + cc] = b0 ? tcol[r] : tcol[r] * bc;
+                    tcol[r] *= bc;
+                }
+            }
+            group_sync(bar_id);
+            // (2) all threads: Y = M21 T11, two entries each (M21[r][k] = N[16 + r][k] = at[k][16 + r])
+            if (!*abortp) {
+                const int r = pt >> 3, c = 2 * (pt & 7);
+                float2 y = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < kTile; ++k) {
+                    const float m = at[k * kRs + kTile + r];
+                    y = ffma2(make_float2(m, m), *reinterpret_cast<const float2 *>(at + k * kRs + c), y);
+                }
+                *reinterpret_cast<float2 *>(at + (kTile + r) * kRs + kTile + c) = y;
+            }
+            group_sync(bar_id);
+            // (3) T21 = -M22^-1 Y (M22^-1 is unit lower triangular)
+            if (!*abortp) {
+                const int r = pt >> 3, c = 2 * (pt & 7);
+                float2 t = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < kTile; ++k)
+                    if (k <= r) {
+                        const float u = -at[(kTile + r) * kRs + k];
+                        t = ffma2(make_float2(u, u),
+                                  *reinterpret_cast<const float2 *>(at + (kTile + k) * kRs + kTile + c), t);
+                    }
+                *reinterpret_cast<float2 *>(at + r * kRs + kTile + c) = t;
+            }
+            group_sync(bar_id);
+            // (4) solver warp: T bf16, row c = column c of T (B operand of the Z and P
+            //     products): [T11 col | T21 col] for c < 16, [0 | T22 col] for c >= 16
+            if (pw == solve_w && !*abortp) {
+                const bool lo = lane < 16;
+                float hi[kTile];
+#pragma unroll
+                for (int r = 0; r < kTile; ++r) hi[r] = lo ? at[r * kRs + kTile + lane] : tcol[r];
+#pragma unroll
+                for (int kg = 0; kg < 2; ++kg) {
                     uint4 w;
-                    w.x = pack_bf16(t[8 * kg], t[8 * kg + 1]);
-                    w.y = pack_bf16(t[8 * kg + 2], t[8 * kg + 3]);
-                    w.z = pack_bf16(t[8 * kg + 4], t[8 * kg + 5]);
-                    w.w = pack_bf16(t[8 * kg + 6], t[8 * kg + 7]);
-                    *reinterpret_cast<uint4 *>(scr + SC_TB + core32_off(c, 8 * kg)) = w;
+                    w.x = lo ? pack_bf16(tcol[8 * kg], tcol[8 * kg + 1]) : 0u;
+                    w.y = lo ? pack_bf16(tcol[8 * kg + 2], tcol[8 * kg + 3]) : 0u;
+                    w.z = lo ? pack_bf16(tcol[8 * kg + 4], tcol[8 * kg + 5]) : 0u;
+                    w.w = lo ? pack_bf16(tcol[8 * kg + 6], tcol[8 * kg + 7]) : 0u;
+                    *reinterpret_cast<uint4 *>(scr + SC_TB + core32_off(lane, 8 * kg)) = w;
+                    uint4 v;
+                    v.x = pack_bf16(hi[8 * kg], hi[8 * kg + 1]);
+                    v.y = pack_bf16(hi[8 * kg + 2], hi[8 * kg + 3]);
+                    v.z = pack_bf16(hi[8 * kg + 4], hi[8 * kg + 5]);
+                    v.w = pack_bf16(hi[8 * kg + 6], hi[8 * kg + 7]);
+                    *reinterpret_cast<uint4 *>(scr + SC_TB + core32_off(lane, 16 + 8 * kg)) = v;
                 }
                 fence_proxy_async_smem();
             }
@@ -894,9 +946,11 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 const int kb = pw & 1, cc = 2 * lane, r0 = 16 * (pw >> 1);
                 const float2 ep = *reinterpret_cast<const float2 *>(sm + SM_EPS + sl * 512 + 4 * (64 * kb + cc));
                 unsigned char *tk = slot + (kb ? SL_K1 : SL_K0), *tq = slot + (kb ? SL_Q1 : SL_Q0);
+                const uint32_t cbase = (uint32_t)r0 * 128u + (uint32_t)(lane & 3) * 4u;
+                const uint32_t chunk = (uint32_t)(lane >> 2);
 #pragma unroll
                 for (int rr = 0; rr < kTile; ++rr) {
-                    const uint32_t o = sw128_off(r0 + rr, cc);
+                    const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
                     const float2 kv = fmul2(bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(tk + o)), ep);
                     const float2 qv = fmul2(bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(tq + o)), ep);
                     *reinterpret_cast<uint32_t *>(tk + o) = pack_bf16(kv.x, kv.y);
