@@ -381,8 +381,10 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_o,
                        const Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte alignment for the 128-byte-swizzled tiles, as an offset into
+    // the shared array, so that every access below stays a shared-memory
+    // access with 32-bit addressing
+    unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     __shared__ Barriers bars;
     volatile int *abortp = &bars.abort_flag;
 
