@@ -289,13 +289,15 @@ __device__ __forceinline__ float rcp(float x) {
     return y;
 }
 
-// Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
+// Warp-uniform bounded wait: every lane polls the barrier and the warp
+// agrees on the outcome (a wait counts as completed only if it completed for
+// all lanes).  Polling from one lane and broadcasting its result leaves that
+// lane in a convergence group of its own after the loop, and the warp then
+// issues each later instruction twice, once per group.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort, unsigned long long limit) {
-    bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    return ok;
+    const bool ok = mbar_wait(bar, parity, abort, limit);
+    return __all_sync(0xffffffffu, ok);
 }
 
 __device__ __forceinline__ void fail(Barriers &bars) {
