@@ -596,18 +596,19 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 KDA_TR(TR_SCAN_ISSUE, c);
                 tc_fence_after();
                 KDA_TR(TR_S_FENCE, c);
+                const uint64_t dk = sdesc(slot_u, 16, 1024, kLayoutSW128);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tm + COL_UP, tm + COL_S16 + 8 * kk,
-                           sdesc(slot_u + (kk >> 2) * SL_K1 + (kk & 3) * 32, 16, 1024, kLayoutSW128),
-                           id1, kk > 0);
+                           sdesc_at(dk, (kk >> 2) * SL_K1 + (kk & 3) * 32), id1, kk > 0);
                 tc_commit(&bars.mma1_done);
                 KDA_TR(TR_S_ISSUED, c);
                 if (!ch.v_zero) {
+                    const uint64_t dv = sdesc(slot_u + SL_V0, SL_V1 - SL_V0, 1024, kLayoutSW128);
+                    const uint64_t db = sdesc(slot_u + SL_B2, 128, 512, kLayoutNone);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
-                        mma_ss(tm + COL_O, sdesc(slot_u + SL_V0 + 2048 * kk, SL_V1 - SL_V0, 1024, kLayoutSW128),
-                               sdesc(slot_u + SL_B2 + 256 * kk, 128, 512, kLayoutNone), id2v, 1);
+                        mma_ss(tm + COL_O, sdesc_at(dv, 2048 * kk), sdesc_at(db, 256 * kk), id2v, 1);
                 }
                 issued = true;
             }
@@ -640,21 +641,23 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             if (tid == 0 && !*abortp) {
                 KDA_TR(TR_SCAN_U, c);
                 tc_fence_after();
+                const uint64_t db = sdesc(slot_u + SL_B2, 128, 512, kLayoutNone);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_ts(tm + COL_O, tm + COL_UN + 8 * kk,
-                           sdesc(slot_u + SL_B2 + 256 * kk, 128, 512, kLayoutNone), id2, 1);
+                    mma_ts(tm + COL_O, tm + COL_UN + 8 * kk, sdesc_at(db, 256 * kk), id2, 1);
                 tc_commit(&bars.d_done);
             }
             store_o();                      // outputs of step c - 1, during the MMA2 round trip
+            // the next step's operands: usually prepared well before MMA2 completes,
+            // so this wait runs during the round trip
+            const bool has_next = c + 1 < nS;
+            bool ready = true;
+            if (has_next) ready = warp_wait(&bars.b_ready[(c + 1) % kPrep], ((c + 1) / kPrep) & 1, abortp, p.wait_limit);
+            if (!ready) fail(bars);
             // ---- step done: outputs, next step's operands (or the final state)
             if (warp_wait(&bars.d_done, c & 1, abortp, p.wait_limit)) {
                 tc_fence_after();
                 if (tid == 0) KDA_TR(TR_SCAN_DONE, c);
-                const bool has_next = c + 1 < nS;
-                bool ready = true;
-                if (has_next) ready = warp_wait(&bars.b_ready[(c + 1) % kPrep], ((c + 1) / kPrep) & 1, abortp, p.wait_limit);
-                if (!ready) fail(bars);
                 if (tid == 0) KDA_TR(TR_S_BR, c);
                 const int sn = (c + 1) % kSlots;
                 const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA + sn * 512);
@@ -780,13 +783,12 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             if (iss && !*abortp) {
                 KDA_TR(TR_PREP_P1, s);
                 tc_fence_after();
+                const uint64_t da = sdesc(slot_u, 16, 1024, kLayoutSW128);
+                const uint64_t dg = sdesc(slot_u + SL_G0, 16, 1024, kLayoutSW128);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a = sdesc(slot_u + (kk >> 2) * SL_K1 + (kk & 3) * 32, 16, 1024, kLayoutSW128);
-                    const uint64_t b = sdesc(slot_u + SL_G0 + (kk >> 2) * (SL_G1 - SL_G0) + (kk & 3) * 32,
-                                             16, 1024, kLayoutSW128);
-                    mma_ss(tP, a, b, idA, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tP, sdesc_at(da, (kk >> 2) * SL_K1 + (kk & 3) * 32),
+                           sdesc_at(dg, (kk >> 2) * (SL_G1 - SL_G0) + (kk & 3) * 32), idA, kk > 0);
                 tc_commit(&bars.a_done[pg]);
                 issued = true;
             }
@@ -934,14 +936,15 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             if (iss && !*abortp) {
                 KDA_TR(TR_PREP_T, s);
                 tc_fence_after();
+                const uint64_t dh = sdesc(slot_u + SL_G0, SL_G1 - SL_G0, 1024, kLayoutSW128);
+                const uint64_t dt = sdesc(scr_u + SC_TB, 128, 512, kLayoutNone);
+                const uint64_t dq = sdesc(scr_u + SC_AQ, 128, 512, kLayoutNone);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_ss(tP, sdesc(slot_u + SL_G0 + 2048 * kk, SL_G1 - SL_G0, 1024, kLayoutSW128),
-                           sdesc(scr_u + SC_TB + 256 * kk, 128, 512, kLayoutNone), idZ, kk > 0);
+                    mma_ss(tP, sdesc_at(dh, 2048 * kk), sdesc_at(dt, 256 * kk), idZ, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk)
-                    mma_ss(tP + 32, sdesc(scr_u + SC_AQ + 256 * kk, 128, 512, kLayoutNone),
-                           sdesc(scr_u + SC_TB + 256 * kk, 128, 512, kLayoutNone), idA, kk > 0);
+                    mma_ss(tP + 32, sdesc_at(dq, 256 * kk), sdesc_at(dt, 256 * kk), idA, kk > 0);
                 tc_commit(&bars.z_done[pg]);
             }
             // ---------------- Ke = Kr Diag(eps), Qe = Qr Diag(eps) in place (the A_kk /

@@ -317,6 +317,15 @@ __host__ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo,
     return d;
 }
 
+// The descriptor d moved by `off` bytes (a multiple of 16).  The start
+// address field is the low 14 bits (address / 16) and every shared-memory
+// address stays below 2^18, so adding to the low word never carries out of
+// the field.
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t d, uint32_t off) {
+    const uint32_t lo = (uint32_t)d + (off >> 4);
+    return ((d >> 32) << 32) | lo;
+}
+
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn,
                                                   bool b_neg = false) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_neg ? 1u : 0u) << 14) |
