@@ -372,6 +372,28 @@ __device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane,
     }
 }
 
+// The last, partial step of a sequence: out of line, so that its code stays
+// out of the instruction stream of the steady-state loop.
+__device__ __noinline__ void gate_pass_partial(unsigned char *slot, int pw, int lane, int Ls,
+                                               float *eps_out, float *dlt_out) {
+    gate_pass<false>(slot, pw, lane, Ls, eps_out, dlt_out);
+}
+
+// Masked plain stores of the last, partial step's outputs (out of line).
+struct OutRegs {
+    uint32_t v[kStep];
+};
+__device__ __noinline__ void store_o_partial(__nv_bfloat16 *dst, size_t step, int Lc, OutRegs ov) {
+#pragma unroll 1
+    for (int r = 0; r < Lc; ++r) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov.v[r]));
+}
+
+// One quarter (32 key channels) of the final state of a chain (out of line).
+__device__ __noinline__ void store_state_quarter(float *dst, OutRegs sv) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) dst[(size_t)i * kD] = __uint_as_float(sv.v[i]);
+}
+
 // kGate: the fused output gate o * sigmoid(z) (p.z), compiled only into the
 // gated instantiation so that the plain operator carries no trace of it.
 template <bool kGate>
@@ -568,10 +590,10 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 o_staged = o_step;
             } else {
                 __nv_bfloat16 *dst = p.o + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
-                const size_t step = (size_t)p.H * kD;
+                OutRegs orr;
 #pragma unroll
-                for (int r = 0; r < kStep; ++r)
-                    if (r < Lc) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov[r]));
+                for (int r = 0; r < kStep; ++r) orr.v[r] = ov[r];
+                store_o_partial(dst, (size_t)p.H * kD, Lc, orr);
             }
             o_step = -1;
         };
@@ -689,9 +711,10 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                         tmem_st16(tm + la + COL_S + 32 * qt + 16, *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
                         if (tid == 0) KDA_TR(qt == 1 ? TR_S_H0 : TR_S_H1, c);
                     } else if (ch.hT) {
-                        float *dst = ch.hT + (size_t)(32 * qt) * kD + j;
+                        OutRegs srr;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) dst[(size_t)i * kD] = __uint_as_float(sv[i]);
+                        for (int i = 0; i < 32; ++i) srr.v[i] = sv[i];
+                        store_state_quarter(ch.hT + (size_t)(32 * qt) * kD + j, srr);
                     }
                 }
                 tmem_ld32(tm + la + COL_O, ov);
@@ -774,7 +797,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             if (ok) {
                 float *eps_out = reinterpret_cast<float *>(sm + SM_EPS + sl * 512);
                 if (Ls == kStep) gate_pass<true>(slot, pw, lane, Ls, eps_out, dlt);
-                else gate_pass<false>(slot, pw, lane, Ls, eps_out, dlt);
+                else gate_pass_partial(slot, pw, lane, Ls, eps_out, dlt);
             }
             fence_proxy_async_smem();
             group_sync(bar_id);                                             // operands written
