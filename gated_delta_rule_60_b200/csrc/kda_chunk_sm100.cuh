@@ -638,6 +638,8 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             // request step c - 1 + kSlots (overlaps the MMA1 round trip)
             if (loader && c >= 1 && c - 1 + kSlots < nS && !*abortp) load_step(c - 1 + kSlots);
             if (prefetcher && c >= 1 && c - 1 + 2 * kSlots < nS) prefetch_step(c - 1 + 2 * kSlots);
+            // outputs of step c - 1, during the MMA1 round trip (thread 0 after its issue)
+            store_o();
             // ---- -(Ke S)^T in bf16: A operand of the second half of MMA2
             if (warp_wait(&bars.mma1_done, c & 1, abortp, p.wait_limit)) {
                 if (tid == 0) KDA_TR(TR_S_M1, c);
@@ -669,7 +671,6 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                     mma_ts(tm + COL_O, tm + COL_UN + 8 * kk, sdesc_at(db, 256 * kk), id2, 1);
                 tc_commit(&bars.d_done);
             }
-            store_o();                      // outputs of step c - 1, during the MMA2 round trip
             // the next step's operands: usually prepared well before MMA2 completes,
             // so this wait runs during the round trip
             const bool has_next = c + 1 < nS;
