@@ -323,7 +323,10 @@ __host__ __device__ __forceinline__ uint32_t core32_off(uint32_t n, uint32_t k) 
 // of the sequence (no masking).  Writes eps (first tile) or delta (second).
 // The cumulative log-decay is summed in base 2 (b = sum of -5 log2(e)
 // sigmoid(g)), so each element costs two MUFU operations for the sigmoid
-// and two for e^{b-m} and its reciprocal.
+// and two for e^{b-m} and its reciprocal.  The first tile's threads sum
+// their tile once ahead (m = b_15) so that the main pass is a single loop;
+// the loops stay rolled by half, which keeps the prep warps' code small
+// enough to share the instruction cache with the scan.
 template <bool kFull>
 __device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane, int Ls,
                                           float *eps_out, float *dlt_out) {
@@ -338,28 +341,33 @@ __device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane,
     const float2 c1 = make_float2(-kLog2e, -kLog2e);
     const float2 c5 = make_float2(-5.f * kLog2e, -5.f * kLog2e);
     const float2 one = make_float2(1.f, 1.f);
-    float2 bb[kTile];
-    float2 b = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int rr = 0; rr < kTile; ++rr) {
-        const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
-        const float2 g = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(slot + oG + o));
-        const float2 x = fmul2(g, c1);
-        const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), one);
-        const float2 sg = make_float2(rcp(den.x), rcp(den.y));              // sigmoid(g)
-        if (kFull || r0 + rr < Ls) b = ffma2(sg, c5, b);
-        bb[rr] = b;
+    // first tile: m = b_15, summed first (the same sums as the main loop)
+    float2 m = make_float2(0.f, 0.f);
+    if (th == 0) {
+#pragma unroll 8
+        for (int rr = 0; rr < kTile; ++rr) {
+            const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
+            const float2 g = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(slot + oG + o));
+            const float2 x = fmul2(g, c1);
+            const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), one);
+            const float2 sg = make_float2(rcp(den.x), rcp(den.y));
+            if (kFull || r0 + rr < Ls) m = ffma2(sg, c5, m);
+        }
     }
-    const float2 tot = bb[kTile - 1];
-    *reinterpret_cast<float2 *>((th == 0 ? eps_out : dlt_out) + 64 * kb + 2 * lane) =
-        make_float2(ex2(tot.x), ex2(tot.y));
-    // first tile: b - m = b - tot; second tile: b - m = b
-    const float2 nbase = th == 0 ? make_float2(-tot.x, -tot.y) : make_float2(0.f, 0.f);
-#pragma unroll
+    const float2 nbase = make_float2(-m.x, -m.y);
+    float2 b = make_float2(0.f, 0.f);
+#pragma unroll 8
     for (int rr = 0; rr < kTile; ++rr) {
         const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
         const bool live = kFull || r0 + rr < Ls;
-        const float2 dd = fadd2(bb[rr], nbase);
+        {
+            const float2 g = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(slot + oG + o));
+            const float2 x = fmul2(g, c1);
+            const float2 den = fadd2(make_float2(ex2(x.x), ex2(x.y)), one);
+            const float2 sg = make_float2(rcp(den.x), rcp(den.y));
+            if (live) b = ffma2(sg, c5, b);
+        }
+        const float2 dd = fadd2(b, nbase);
         const float2 er = make_float2(ex2(dd.x), ex2(dd.y));                // e^{b-m}
         const float2 ei = make_float2(rcp(er.x), rcp(er.y));                // e^{m-b}
         const uint32_t kraw = live ? *reinterpret_cast<const uint32_t *>(slot + oK + o) : 0u;
@@ -370,6 +378,9 @@ __device__ __forceinline__ void gate_pass(unsigned char *slot, int pw, int lane,
         *reinterpret_cast<uint32_t *>(slot + oQ + o) = pack_bf16(qr.x, qr.y);
         *reinterpret_cast<uint32_t *>(slot + oG + o) = pack_bf16(kh.x, kh.y);
     }
+    // eps (first tile: b_15 = m) or delta (second tile: b_31 - b_15)
+    *reinterpret_cast<float2 *>((th == 0 ? eps_out : dlt_out) + 64 * kb + 2 * lane) =
+        make_float2(ex2(b.x), ex2(b.y));
 }
 
 // The last, partial step of a sequence: out of line, so that its code stays
@@ -979,7 +990,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 unsigned char *tk = slot + (kb ? SL_K1 : SL_K0), *tq = slot + (kb ? SL_Q1 : SL_Q0);
                 const uint32_t cbase = (uint32_t)r0 * 128u + (uint32_t)(lane & 3) * 4u;
                 const uint32_t chunk = (uint32_t)(lane >> 2);
-#pragma unroll
+#pragma unroll 8
                 for (int rr = 0; rr < kTile; ++rr) {
                     const uint32_t o = cbase + (rr >> 3) * 1024u + (rr & 7) * 128u + ((chunk ^ (rr & 7)) << 4);
                     const float2 kv = fmul2(bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(tk + o)), ep);
