@@ -277,6 +277,13 @@ __device__ __forceinline__ int longest_first_cta(const Params &p, int tid) {
     return pick * p.H + (int)(blockIdx.x % p.H);
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -840,25 +847,26 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (warp_wait(&bars.a_done[pg], par, abortp, p.wait_limit)) {
                     if (pt == 0) KDA_TR(TR_PREP_A, s);
                     tc_fence_after();
-                    uint32_t d[32];
-                    tmem_ld32(tPl, d);
-                    tmem_wait_ld();
-                    __syncwarp();
                     const int r = lane;
-                    if (pw == 0) {
-                        const float bl = bars.beta_s[pg][r];
-                        float *at = reinterpret_cast<float *>(scr + SC_AT);
+                    const float bl = bars.beta_s[pg][r];
+                    float *at = reinterpret_cast<float *>(scr + SC_AT);
+#pragma unroll 1
+                    for (int kg = 0; kg < 4; ++kg) {
+                        uint32_t d[8];
+                        tmem_ld8(tPl + 8 * kg, d);
+                        tmem_wait_ld();
+                        if (pw == 0) {
 #pragma unroll
-                        for (int i = 0; i < kStep; ++i)
-                            at[i * (kScRow / 4) + r] = i < r ? bl * __uint_as_float(d[i]) : 0.f;
-                    } else {
-#pragma unroll
-                        for (int kg = 0; kg < 4; ++kg) {
+                            for (int t = 0; t < 8; ++t) {
+                                const int i = 8 * kg + t;
+                                at[i * (kScRow / 4) + r] = i < r ? bl * __uint_as_float(d[t]) : 0.f;
+                            }
+                        } else {
                             float x[8];
 #pragma unroll
                             for (int t = 0; t < 8; ++t) {
                                 const int i = 8 * kg + t;
-                                x[t] = i <= r ? __uint_as_float(d[i]) : 0.f;
+                                x[t] = i <= r ? __uint_as_float(d[t]) : 0.f;
                             }
                             uint4 w;
                             w.x = pack_bf16(x[0], x[1]);
