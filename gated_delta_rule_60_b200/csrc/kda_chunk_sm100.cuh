@@ -19,8 +19,9 @@
 //   A_kk = Kr Kh^T,  A_qk = Qr Kh^T   (causal entries are e^{b_r - b_i} <= 1)
 //   T = (I + Diag(beta) strict_lower(A_kk))^-1 Diag(beta)     (32 x 32)
 //   P = causal(A_qk) T,   Z = Diag(delta) Kh^T T              (d_k x 32)
-// (T by forward substitution on the CUDA cores; every product on the tensor
-// cores.)
+// (T on the CUDA cores, by 16 x 16 blocks: forward substitution inside the
+// diagonal blocks, two small products for the off-diagonal one; every
+// product of the step on the tensor cores.)
 // With Ke = Kr Diag(eps) = K e^b and Qe = Q e^b the step is exactly
 //   W = V - Ke S0,   S_next = Diag(gamma) S0 + Z W,   O = Qe S0 + P W.
 // On the tensor cores everything is transposed so that the 128 value
@@ -49,6 +50,16 @@
 // through mbarriers.  Every mbarrier wait is bounded; a wait that runs out
 // raises the device status word, makes the CTA drain its own copies and
 // MMAs, free its tensor memory and return.
+//
+// What sets the speed.  The scan's chain per step is: MMA1 issue (eight
+// tcgen05.mma from one thread), MMA1 round trip, -U, MMA2 issue and round
+// trip, the state pass.  The prep warpgroups keep ahead of it, but they
+// share every SM sub-partition with a scan warp, so their instruction count
+// and, above all, their code size matter: sixteen warps running four roles
+// of one large loop contend for the instruction cache.  Hence every wait is
+// polled by all lanes (a warp never splits into two issue groups), cold paths
+// (partial steps, the final state) are out of line, and the prep's element
+// loops are rolled where no register array forces full unrolling.
 #pragma once
 
 #include "kda_common.cuh"
