@@ -177,6 +177,7 @@ struct Params {
     long T_tot;
     int mode, G;
     long seg_len;
+    long seg0_len;
     float *ws_R, *ws_M, *ws_S;    // [G][H][128][128] each (segment modes)
     unsigned long long wait_limit;  // bound of a pipeline wait, SM clock cycles
     int stall_step;               // diagnostic: step at which the scan waits on `never` (-1: none)
@@ -221,8 +222,15 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
     c.ok = seq_bounds(p.cu, 0, 1, p.T_tot, b0, b1);
     int s;
     if (p.mode == kModeSegLocal && cta < p.H * p.G) {
-        c.h = cta / p.G;
-        s = cta % p.G;
+        // segment 0 of every head first (the longest runs start first), then
+        // segments 1 .. G-1
+        if (cta < p.H) {
+            c.h = cta;
+            s = 0;
+        } else {
+            c.h = (cta - p.H) / (p.G - 1);
+            s = 1 + (cta - p.H) % (p.G - 1);
+        }
         c.h0 = (s == 0 && p.h0) ? p.h0 + (size_t)c.h * kSt : nullptr;
         c.hT = (s == 0 ? p.ws_S + ((size_t)1 * p.H + c.h) * kSt
                        : p.ws_R + ((size_t)s * p.H + c.h) * kSt);
@@ -242,9 +250,12 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
         c.h0 = p.ws_S + ((size_t)s * p.H + c.h) * kSt;
         c.hT = (s == p.G - 1 && p.hT) ? p.hT + (size_t)c.h * kSt : nullptr;
     }
-    c.start = (int64_t)s * p.seg_len;
+    // segment 0 covers [0, seg0_len); segment s >= 1 starts at
+    // seg0_len + (s - 1) seg_len (the last one may be shorter)
+    c.start = s == 0 ? 0 : (int64_t)p.seg0_len + (int64_t)(s - 1) * p.seg_len;
     const int64_t rem = p.T_tot - c.start;
-    c.L = (int)(rem < p.seg_len ? rem : p.seg_len);
+    const long len = s == 0 ? p.seg0_len : p.seg_len;
+    c.L = (int)(rem < len ? (rem < 0 ? 0 : rem) : len);
     if (!c.ok) {
         c.L = 0;
         c.hT = nullptr;
@@ -1179,24 +1190,47 @@ inline int sm_count() {
 // H*(2G-1) chains and the final pass H*(G-1), each over T/G tokens.
 struct SegPlan {
     int G;
-    long seg_len;
+    long seg_len;      // segments 1 .. G-1
+    long seg0_len;     // segment 0: a whole multiple of seg_len
 };
 
+// Segments for one long sequence per head.  The local pass runs segment 0
+// (final after it) and, for each later segment, one run from zero and one
+// from the identity; the final pass re-runs the later segments.  Segment 0 is
+// k times as long as the others: its H runs start first on H SMs while the
+// other SMs work through the 2 H (G - 1) short runs, which evens out the
+// local pass's last wave.  Cost model, in units of one short run: local =
+// k + ceil(r / sms) with r the short runs left after k of them per free SM
+// (or ceil(n / (sms - H)) when none are left), final = ceil(H (G-1) / sms);
+// minimised over G and k per token of the sequence.
 inline SegPlan plan_segments(int N, int64_t T, int H) {
-    SegPlan pl{1, (long)T};
+    SegPlan pl{1, (long)T, (long)T};
     if (N != 1 || T < 8192) return pl;
     const int sms = sm_count();
     double best = (double)((H + sms - 1) / sms);
-    for (int G = 2; G <= 64; ++G) {
-        const long seg = (long)(((T + G - 1) / G + 31) / 32 * 32);
-        if (seg < 4096) break;
-        if ((T + seg - 1) / seg != G) continue;
-        const int w1 = (H * (2 * G - 1) + sms - 1) / sms;
-        const int w3 = (H * (G - 1) + sms - 1) / sms;
-        const double cost = (double)(w1 + w3) / G;
-        if (cost < 0.9 * best) {
-            best = cost;
-            pl = SegPlan{G, seg};
+    for (int k = 1; k <= 3; ++k) {
+        for (int G = 2; G <= 64; ++G) {
+            const long seg = (long)(((T + (k + G - 1) - 1) / (k + G - 1) + 31) / 32 * 32);
+            if (seg < 4096) break;
+            const long seg0 = (long)k * seg;
+            const int64_t last = T - seg0 - (int64_t)(G - 2) * seg;      // length of segment G - 1
+            if (last <= 0 || last > seg) continue;
+            const long n = 2L * H * (G - 1);
+            double local;
+            if (H >= sms) {
+                local = (double)((H * (long)k + n + sms - 1) / sms);
+            } else {
+                const long early = (long)k * (sms - H);
+                const long r = n > early ? n - early : 0;
+                local = r > 0 ? (double)k + (double)((r + sms - 1) / sms)
+                              : (double)std::max<long>(k, (n + (sms - H) - 1) / (sms - H));
+            }
+            const double fin = (double)((H * (long)(G - 1) + sms - 1) / sms);
+            const double cost = (local + fin) * (double)seg / (double)T;
+            if (cost < 0.97 * best) {
+                best = cost;
+                pl = SegPlan{G, seg, seg0};
+            }
         }
     }
     return pl;
@@ -1251,6 +1285,7 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.mode = prefill::kModeChains;
     p.G = 1;
     p.seg_len = (long)T_tot;
+    p.seg0_len = (long)T_tot;
     p.ws_R = p.ws_M = p.ws_S = nullptr;
     p.stall_step = debug_stall().step.exchange(-1);
     const unsigned long long lim = debug_stall().limit.exchange(0);
@@ -1265,6 +1300,7 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     float *ws = static_cast<float *>(workspace);
     p.G = pl.G;
     p.seg_len = pl.seg_len;
+    p.seg0_len = pl.seg0_len;
     p.ws_R = ws;
     p.ws_M = ws + per;
     p.ws_S = ws + 2 * per;

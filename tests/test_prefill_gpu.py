@@ -234,6 +234,18 @@ def test_long_sequence_segmented():
     check(inp, o, hT)
 
 
+def test_long_sequence_segmented_long_first_segment():
+    """A shape whose segment plan gives segment 0 twice the length of the
+    others on a 148-SM part (16 heads, 50,000 tokens: nine segments, the last
+    one ragged), with a carried state; every unit checked against the
+    oracle."""
+    T, H = 50000, 16
+    assert binding.kda_chunk_fwd_workspace_size(1, T, H, 128, 128, torch.bfloat16) > 0
+    inp = inputs.make_prefill([T], H, 128, 128, torch.bfloat16, seed=97, h0_std=0.02)
+    o, hT = run(inp)
+    check(inp, o, hT)
+
+
 def test_long_1m_workload_sampled():
     """The long-context workload (T = 1,048,576, H = 16, bf16, S0 = 0): the
     oracle runs 2 seeded heads over the full length."""
