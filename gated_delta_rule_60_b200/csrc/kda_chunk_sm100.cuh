@@ -154,17 +154,19 @@ struct Barriers {
     int abort_flag;
 };
 
-// Launch modes.  kModeChains: one CTA per (sequence, head).  The two
-// segment modes split one long sequence per head into G segments of seg_len
-// tokens (the state recurrence is linear in (S0, V), so
-// S_end = M_s S_start + R_s):
-//   kModeSegLocal: CTAs [0, H*G) run every segment from a zero state (the
-//     real h0 for segment 0) giving R_s (segment 0's run is final: it writes
-//     o and the start state of segment 1); CTAs [H*G, H*(2G-1)) run segments
-//     s >= 1 with v = 0 from the identity, giving the transfer matrix M_s.
-//   kModeSegFinal: CTAs [0, H*(G-1)) re-run segments s >= 1 from their true
-//     start states (combined in between) and write o, and hT at the end.
-enum { kModeChains = 0, kModeSegLocal = 1, kModeSegFinal = 2 };
+// Launch modes.  kModeChains: one CTA per (sequence, head).  kModeSegLocal
+// splits one long sequence per head into G segments (segment 0 of seg0_len
+// tokens, the others of seg_len).  The recurrence is linear in (S0, V): from
+// a start state S_start a segment ends in M_s S_start + R_s and its outputs
+// are o_t = o_t(zero start) + S_start^T (M_{s,t}^T q_t), with M_{s,t} the
+// transfer from the segment start to token t.  CTAs [0, H*G) run segment 0
+// from the real h0 (final: o and the start state of segment 1) and the later
+// segments from zero (R_s, and their zero-start outputs into o); CTAs
+// [H*G, H*(2G-1)) run the later segments from the identity with v = 0 (M_s,
+// and M_{s,t}^T q_t into a scratch).  seg_combine_kernel then forms the start
+// states and the final state, and seg_correct_kernel adds S_start^T times the
+// scratch to the outputs of every later segment.
+enum { kModeChains = 0, kModeSegLocal = 1 };
 
 struct Params {
     const __nv_bfloat16 *beta;
@@ -172,6 +174,7 @@ struct Params {
     const float *h0;
     const int32_t *cu;
     __nv_bfloat16 *o;
+    __nv_bfloat16 *om;            // segment modes: outputs of the identity runs, rows from seg0_len
     float *hT;
     int N, H;
     long T_tot;
@@ -195,6 +198,8 @@ struct Chain {
     float *hT;               // nullptr = do not write the final state
     bool write_o;
     bool v_zero;             // treat v as zero (transfer-matrix runs)
+    bool o_alt;              // write o to the identity-run scratch (Params::om)
+    bool gate;               // apply the output gate (gated launches)
 };
 
 __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
@@ -202,6 +207,8 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
     c.h0_identity = false;
     c.v_zero = false;
     c.write_o = true;
+    c.o_alt = false;
+    c.gate = true;
     constexpr size_t kSt = (size_t)kD * kD;
     if (p.mode == kModeChains) {
         const int n = cta / p.H;
@@ -221,9 +228,10 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
     int64_t b0 = 0, b1 = 0;
     c.ok = seq_bounds(p.cu, 0, 1, p.T_tot, b0, b1);
     int s;
-    if (p.mode == kModeSegLocal && cta < p.H * p.G) {
-        // segment 0 of every head first (the longest runs start first), then
-        // segments 1 .. G-1
+    if (cta < p.H * p.G) {
+        // runs from the real start state (segment 0, final) or from zero (later
+        // segments); segment 0 of every head first, so that the longest runs
+        // start first
         if (cta < p.H) {
             c.h = cta;
             s = 0;
@@ -234,21 +242,19 @@ __device__ __forceinline__ Chain chain_of(const Params &p, int cta) {
         c.h0 = (s == 0 && p.h0) ? p.h0 + (size_t)c.h * kSt : nullptr;
         c.hT = (s == 0 ? p.ws_S + ((size_t)1 * p.H + c.h) * kSt
                        : p.ws_R + ((size_t)s * p.H + c.h) * kSt);
-        c.write_o = s == 0;
-    } else if (p.mode == kModeSegLocal) {
+        c.gate = s == 0;          // later segments are gated after their correction
+    } else {
+        // runs from the identity with v = 0: the transfer matrix M_s (final
+        // state) and M_{s,t}^T q_t (outputs, to the scratch)
         const int i = cta - p.H * p.G;
         c.h = i / (p.G - 1);
         s = 1 + i % (p.G - 1);
         c.h0 = nullptr;
         c.h0_identity = true;
         c.v_zero = true;
-        c.write_o = false;
+        c.o_alt = true;
+        c.gate = false;
         c.hT = p.ws_M + ((size_t)s * p.H + c.h) * kSt;
-    } else {
-        c.h = cta / (p.G - 1);
-        s = 1 + cta % (p.G - 1);
-        c.h0 = p.ws_S + ((size_t)s * p.H + c.h) * kSt;
-        c.hT = (s == p.G - 1 && p.hT) ? p.hT + (size_t)c.h * kSt : nullptr;
     }
     // segment 0 covers [0, seg0_len); segment s >= 1 starts at
     // seg0_len + (s - 1) seg_len (the last one may be shorter)
@@ -443,6 +449,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_v,
                        const __grid_constant__ CUtensorMap map_g,
                        const __grid_constant__ CUtensorMap map_o,
+                       const __grid_constant__ CUtensorMap map_om,
                        const Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled tiles, as an offset into
@@ -602,7 +609,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         auto store_o = [&]() {
             if (o_step < 0 || !ch.write_o) { o_step = -1; return; }
             const int Lc = L - kStep * o_step;
-            if (kGate) {
+            if (kGate && ch.gate) {
                 // fused output gate: o * sigmoid(z) on the values in registers
                 const __nv_bfloat16 *zr = p.z + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
                 const size_t step = (size_t)p.H * kD;
@@ -629,7 +636,9 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 fence_proxy_async_smem();
                 o_staged = o_step;
             } else {
-                __nv_bfloat16 *dst = p.o + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
+                __nv_bfloat16 *dst =
+                    ch.o_alt ? p.om + ((size_t)(start - p.seg0_len + kStep * o_step) * p.H + h) * kD + j
+                             : p.o + ((size_t)(start + kStep * o_step) * p.H + h) * kD + j;
                 OutRegs orr;
 #pragma unroll
                 for (int r = 0; r < kStep; ++r) orr.v[r] = ov[r];
@@ -641,9 +650,11 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
         auto flush_o = [&]() {
             if (!o_issuer || o_staged <= o_stored) return;
             const unsigned char *st = sm + SM_OST + (o_staged & 1) * kOstBytes;
-            const int z = (int)(start + (int64_t)kStep * o_staged);
-            tma_store_3d(&map_o, st, 0, h, z);
-            tma_store_3d(&map_o, st + 4096, 64, h, z);
+            // the identity runs' scratch holds rows from seg0_len on
+            const int z = (int)(start + (int64_t)kStep * o_staged - (ch.o_alt ? p.seg0_len : 0));
+            const CUtensorMap *mp = ch.o_alt ? &map_om : &map_o;
+            tma_store_3d(mp, st, 0, h, z);
+            tma_store_3d(mp, st + 4096, 64, h, z);
             bulk_commit_group();
             o_stored = o_staged;
         };
@@ -1095,13 +1106,17 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
 #endif
 }
 
-// Segment combine (between the two segment modes): for each head,
-// S_{s+1} = M_s S_s + R_s for s = 1 .. G-2, in fp32, starting from S_1 (the
-// final state of segment 0's run).  One CTA per head; the running state and
-// the current transfer matrix sit in shared memory (128 KB).
+// Segment combine: for each head, S_{s+1} = M_s S_s + R_s for s = 1 .. G-1, in
+// fp32, starting from S_1 (the final state of segment 0's run); S_G is the
+// final state (hT).  One CTA per head; the running state and the current
+// transfer matrix sit in shared memory (128 KB).
 __global__ void __launch_bounds__(256)
 seg_combine_kernel(const float *__restrict__ M, const float *__restrict__ R,
-                   float *__restrict__ S, int H, int G) {
+                   float *__restrict__ S, float *__restrict__ hT, const int32_t *__restrict__ cu,
+                   long T, int H, int G) {
+    // malformed bounds (reported by the local pass): the states were never
+    // written, so nothing is combined
+    if (cu != nullptr && (cu[0] != 0 || (long)cu[1] != T)) return;
     extern __shared__ __align__(16) float shm[];
     float *Sc = shm;               // [128][128]
     float *Ms = shm + kD * kD;     // [128][128]
@@ -1109,7 +1124,7 @@ seg_combine_kernel(const float *__restrict__ M, const float *__restrict__ R,
     constexpr size_t kSt = (size_t)kD * kD;
     for (int e = t; e < kD * kD; e += 256) Sc[e] = S[((size_t)1 * H + h) * kSt + e];
     const int j = t & (kD - 1), i0 = t >> 7;     // column j, rows i0 + 2m
-    for (int s = 1; s <= G - 2; ++s) {
+    for (int s = 1; s <= G - 1; ++s) {
         __syncthreads();
         const float *Mg = M + ((size_t)s * H + h) * kSt;
         for (int e = t; e < kD * kD; e += 256) Ms[e] = Mg[e];
@@ -1124,11 +1139,115 @@ seg_combine_kernel(const float *__restrict__ M, const float *__restrict__ R,
             for (int m = 0; m < kD / 2; ++m) acc[m] = fmaf(Ms[(i0 + 2 * m) * kD + k], skj, acc[m]);
         }
         __syncthreads();
-        float *Sg = S + ((size_t)(s + 1) * H + h) * kSt;
+        // start state of segment s + 1, or the final state after the last one
+        float *Sg = s + 1 < G ? S + ((size_t)(s + 1) * H + h) * kSt : (hT ? hT + (size_t)h * kSt : nullptr);
 #pragma unroll
         for (int m = 0; m < kD / 2; ++m) {
             Sc[(i0 + 2 * m) * kD + j] = acc[m];
-            Sg[(size_t)(i0 + 2 * m) * kD + j] = acc[m];
+            if (Sg) Sg[(size_t)(i0 + 2 * m) * kD + j] = acc[m];
+        }
+    }
+}
+
+// Segment correction: o_t <- o_t + S_start(s)^T om_t for the tokens t of every
+// segment s >= 1 (om_t = M_{s,t}^T q_t from the identity run), then the output
+// gate when one is given.  Per (segment, head) this is the product
+// [tokens x 128] x [128 x 128] with the start state as the right factor; it
+// reads and writes each output once and is bound by HBM (about 43 flops per
+// byte), so the warp-level bf16 MMA with fp32 accumulation serves.  CTA: 8
+// warps, 128 tokens a tile (16 per warp), kCorTiles tiles; the start state
+// (transposed, bf16) and the tile sit in shared memory in rows padded to 272
+// bytes, so that each 8 x 8 matrix load touches all banks once.
+constexpr int kCorThreads = 256;
+constexpr int kCorTile = 128;
+constexpr int kCorTiles = 8;
+constexpr int kCorRow = 136;                     // bf16 per padded shared-memory row
+constexpr int kCorSmem = 2 * 128 * kCorRow * 2;  // start state and one tile
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kCorThreads)
+seg_correct_kernel(const float *__restrict__ S, const __nv_bfloat16 *__restrict__ om,
+                   __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ z,
+                   const int32_t *__restrict__ cu, int H, long T, long seg_len, long seg0_len) {
+    // malformed bounds (reported by the local pass): nothing to correct
+    if (cu != nullptr && (cu[0] != 0 || (long)cu[1] != T)) return;
+    extern __shared__ __align__(16) unsigned char cs_raw[];
+    __nv_bfloat16 *sT = reinterpret_cast<__nv_bfloat16 *>(cs_raw);   // [n][k] = S_start[k][n]
+    __nv_bfloat16 *aT = sT + 128 * kCorRow;                          // [token][k] = om
+    const int sg = 1 + (int)blockIdx.z, h = (int)blockIdx.y;
+    const long seg_start = seg0_len + (long)(sg - 1) * seg_len;
+    const long seg_end = seg_start + seg_len < T ? seg_start + seg_len : T;
+    const long t_begin = seg_start + (long)blockIdx.x * (kCorTile * kCorTiles);
+    if (t_begin >= seg_end) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float *Sg = S + ((size_t)sg * H + h) * kD * kD;
+    for (int e = tid; e < kD * kD; e += kCorThreads)
+        sT[(e & (kD - 1)) * kCorRow + (e >> 7)] = __float2bfloat16_rn(Sg[e]);
+    const int g = lane >> 2, tq = lane & 3, rbase = 16 * warp;
+    // this lane's rows of the 8 x 8 matrices: A (tokens x k) and B (n x k)
+    const uint32_t a_addr = smem_u32(aT + (rbase + (lane & 7) + ((lane >> 3) & 1) * 8) * kCorRow +
+                                     (lane >> 4) * 8);
+    const uint32_t b_addr = smem_u32(sT + ((lane & 7) + (lane >> 4) * 8) * kCorRow + ((lane >> 3) & 1) * 8);
+#pragma unroll 1
+    for (int tile = 0; tile < kCorTiles; ++tile) {
+        const long t0 = t_begin + (long)tile * kCorTile;
+        if (t0 >= seg_end) break;
+        __syncthreads();              // the start state is written; the last tile's reads are done
+        for (int c = tid; c < kCorTile * 16; c += kCorThreads) {      // 16-byte chunks, 16 a row
+            const int r = c >> 4, q = c & 15;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (t0 + r < seg_end)
+                v = *reinterpret_cast<const uint4 *>(om + ((size_t)(t0 + r - seg0_len) * H + h) * kD + 8 * q);
+            *reinterpret_cast<uint4 *>(aT + r * kCorRow + 8 * q) = v;
+        }
+        __syncthreads();
+        float acc[16][4];
+#pragma unroll
+        for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(a, a_addr + kk * 32);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t b[4];
+                ldsm_x4(b, b_addr + (np * 16 * kCorRow) * 2 + kk * 32);
+                mma_16816(acc[2 * np], a, b[0], b[1]);
+                mma_16816(acc[2 * np + 1], a, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const long t = t0 + rbase + g + 8 * hf;
+            if (t >= seg_end) continue;
+            __nv_bfloat16 *orow = o + ((size_t)t * H + h) * kD;
+            const __nv_bfloat16 *zrow = z ? z + ((size_t)t * H + h) * kD : nullptr;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                const int n = 8 * nt + 2 * tq;
+                const float2 base = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(orow + n));
+                float x0 = base.x + acc[nt][2 * hf], x1 = base.y + acc[nt][2 * hf + 1];
+                if (zrow) {
+                    const float2 zz = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(zrow + n));
+                    x0 *= out_gate(zz.x);
+                    x1 *= out_gate(zz.y);
+                }
+                *reinterpret_cast<__nv_bfloat162 *>(orow + n) = __floats2bfloat162_rn(x0, x1);
+            }
         }
     }
 }
@@ -1248,17 +1367,20 @@ inline DebugStall &debug_stall() {
     return d;
 }
 
+// Segmented runs: R, M and S states (3 x G x H fp32 128 x 128), then the
+// identity runs' outputs for the tokens after segment 0 (bf16).
 inline size_t sm100_workspace_bytes(int N, int64_t T, int H) {
     const SegPlan pl = plan_segments(N, T, H);
     if (pl.G <= 1) return 0;
-    return 3 * (size_t)pl.G * H * prefill::kD * prefill::kD * sizeof(float);
+    return 3 * (size_t)pl.G * H * prefill::kD * prefill::kD * sizeof(float) +
+           (size_t)(T - pl.seg0_len) * H * prefill::kD * sizeof(__nv_bfloat16);
 }
 
 inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
                                   const void *beta, const float *h0, const int32_t *cu, int N,
                                   int64_t T_tot, int H, const void *z, void *o, float *hT,
                                   void *workspace, cudaStream_t s) {
-    CUtensorMap mq, mk, mv, mg, mo;
+    CUtensorMap mq, mk, mv, mg, mo, mom;
     // With no tokens the token pointers may be NULL and no tile is ever
     // copied (every chain is empty, or malformed and skipped); the maps then
     // describe one row of hT, which the caller passes whenever this runs.
@@ -1287,15 +1409,16 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.seg_len = (long)T_tot;
     p.seg0_len = (long)T_tot;
     p.ws_R = p.ws_M = p.ws_S = nullptr;
+    p.om = nullptr;
     p.stall_step = debug_stall().step.exchange(-1);
     const unsigned long long lim = debug_stall().limit.exchange(0);
     p.wait_limit = (p.stall_step >= 0 && lim > 0) ? lim : prefill::kWaitLimit;
     const SegPlan pl = plan_segments(N, T_tot, H);
     if (pl.G <= 1) {
-        kern<<<(unsigned)(N * H), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);
+        kern<<<(unsigned)(N * H), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, mo, p);
         return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
-    // one long sequence per head: local pass, combine, final pass
+    // one long sequence per head: local pass, combine, correction
     const size_t per = (size_t)pl.G * H * prefill::kD * prefill::kD;
     float *ws = static_cast<float *>(workspace);
     p.G = pl.G;
@@ -1304,17 +1427,26 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.ws_R = ws;
     p.ws_M = ws + per;
     p.ws_S = ws + 2 * per;
+    p.om = reinterpret_cast<__nv_bfloat16 *>(ws + 3 * per);
+    if (!make_qkvg_map(&mom, p.om, H, T_tot - pl.seg0_len)) return KDA_ERR_CUDA;
     p.mode = prefill::kModeSegLocal;
-    kern<<<(unsigned)(H * (2 * pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);
+    kern<<<(unsigned)(H * (2 * pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, mom, p);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     const int comb_smem = 2 * prefill::kD * prefill::kD * (int)sizeof(float);
     if (cudaFuncSetAttribute(prefill::seg_combine_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, comb_smem) != cudaSuccess)
         return KDA_ERR_CUDA;
-    prefill::seg_combine_kernel<<<(unsigned)H, 256, comb_smem, s>>>(p.ws_M, p.ws_R, p.ws_S, H, pl.G);
+    prefill::seg_combine_kernel<<<(unsigned)H, 256, comb_smem, s>>>(p.ws_M, p.ws_R, p.ws_S, hT, cu,
+                                                                   (long)T_tot, H, pl.G);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
-    p.mode = prefill::kModeSegFinal;
-    kern<<<(unsigned)(H * (pl.G - 1)), prefill::kThreads, prefill::kSmemAlloc, s>>>(mq, mk, mv, mg, mo, p);
+    if (cudaFuncSetAttribute(prefill::seg_correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             prefill::kCorSmem) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    const long per_cta = (long)prefill::kCorTile * prefill::kCorTiles;
+    const dim3 cgrid((unsigned)((pl.seg_len + per_cta - 1) / per_cta), (unsigned)H, (unsigned)(pl.G - 1));
+    prefill::seg_correct_kernel<<<cgrid, prefill::kCorThreads, prefill::kCorSmem, s>>>(
+        p.ws_S, p.om, static_cast<__nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(z), cu, H,
+        (long)T_tot, pl.seg_len, pl.seg0_len);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
