@@ -1313,24 +1313,25 @@ struct SegPlan {
     long seg0_len;     // segment 0: a whole multiple of seg_len
 };
 
-// Segments for one long sequence per head.  The local pass runs segment 0
-// (final after it) and, for each later segment, one run from zero and one
-// from the identity; the final pass re-runs the later segments.  Segment 0 is
-// k times as long as the others: its H runs start first on H SMs while the
-// other SMs work through the 2 H (G - 1) short runs, which evens out the
-// local pass's last wave.  Cost model, in units of one short run: local =
-// k + ceil(r / sms) with r the short runs left after k of them per free SM
-// (or ceil(n / (sms - H)) when none are left), final = ceil(H (G-1) / sms);
-// minimised over G and k per token of the sequence.
+// Segments for one long sequence per head.  The local pass is the only pass
+// of serial chains: segment 0 (final after it) and, for each later segment,
+// one run from zero and one from the identity; the combine and the correction
+// after it are short.  Segment 0 may be k times as long as the others: its H
+// runs start first on H SMs while the other SMs work through the 2 H (G - 1)
+// short runs, which can even out the local pass's last wave.  Cost model, in
+// units of one short run: k + ceil(r / sms) with r the short runs left after
+// k of them per free SM (or ceil(n / (sms - H)) when none are left); the plan
+// minimises it per token of the sequence, and among equal costs keeps the
+// fewest segments (a shorter combine, fewer CTAs).
 inline SegPlan plan_segments(int N, int64_t T, int H) {
     SegPlan pl{1, (long)T, (long)T};
     if (N != 1 || T < 8192) return pl;
     const int sms = sm_count();
     double best = (double)((H + sms - 1) / sms);
-    for (int k = 1; k <= 3; ++k) {
-        for (int G = 2; G <= 64; ++G) {
+    for (int G = 2; G <= 64; ++G) {
+        for (int k = 1; k <= 3; ++k) {
             const long seg = (long)(((T + (k + G - 1) - 1) / (k + G - 1) + 31) / 32 * 32);
-            if (seg < 4096) break;
+            if (seg < 4096) continue;
             const long seg0 = (long)k * seg;
             const int64_t last = T - seg0 - (int64_t)(G - 2) * seg;      // length of segment G - 1
             if (last <= 0 || last > seg) continue;
@@ -1344,8 +1345,7 @@ inline SegPlan plan_segments(int N, int64_t T, int H) {
                 local = r > 0 ? (double)k + (double)((r + sms - 1) / sms)
                               : (double)std::max<long>(k, (n + (sms - H) - 1) / (sms - H));
             }
-            const double fin = (double)((H * (long)(G - 1) + sms - 1) / sms);
-            const double cost = (local + fin) * (double)seg / (double)T;
+            const double cost = local * (double)seg / (double)T;
             if (cost < 0.97 * best) {
                 best = cost;
                 pl = SegPlan{G, seg, seg0};

@@ -236,10 +236,10 @@ def test_long_sequence_segmented():
 
 def test_long_sequence_segmented_long_first_segment():
     """A shape whose segment plan gives segment 0 twice the length of the
-    others on a 148-SM part (16 heads, 50,000 tokens: nine segments, the last
+    others on a 148-SM part (12 heads, 52,901 tokens: twelve segments, the last
     one ragged), with a carried state; every unit checked against the
     oracle."""
-    T, H = 50000, 16
+    T, H = 52901, 12
     assert binding.kda_chunk_fwd_workspace_size(1, T, H, 128, 128, torch.bfloat16) > 0
     inp = inputs.make_prefill([T], H, 128, 128, torch.bfloat16, seed=97, h0_std=0.02)
     o, hT = run(inp)
