@@ -340,6 +340,11 @@ __device__ __forceinline__ void fail(Barriers &bars) {
     raise_error(kErrTimeout);
 }
 
+// Diagnostic stall (out of line, off the steady-state instruction stream).
+__device__ __noinline__ void stall_here(Barriers &bars, volatile int *abort, unsigned long long limit) {
+    if (!warp_wait(&bars.never, 0, abort, limit)) fail(bars);
+}
+
 // Barrier among the warps of one warpgroup (id >= 1; 0 is __syncthreads).
 __device__ __forceinline__ void group_sync(int id) {
     asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
@@ -663,7 +668,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             const uint32_t slot_u = s_base + SM_SLOT + sl * kSlotBytes;
             // diagnostic: a wait that nothing completes, so that the bounded
             // wait runs out here and the CTA takes its abort and drain path
-            if (c == p.stall_step && !warp_wait(&bars.never, 0, abortp, p.wait_limit)) fail(bars);
+            if (c == p.stall_step) stall_here(bars, abortp, p.wait_limit);
             // ---- MMA1: [(Ke S)^T | (Qe S)^T] = bf16(S)^T [Ke ; Qe]^T, then the v part of MMA2
             if (tid == 0 && !*abortp) {
                 KDA_TR(TR_SCAN_ISSUE, c);
@@ -735,6 +740,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (tid == 0) KDA_TR(TR_S_BR, c);
                 const int sn = (c + 1) % kSlots;
                 const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA + sn * 512);
+                tmem_ld32(tm + la + COL_O, ov);      // waited for with the first quarter
 #pragma unroll 1
                 for (int qt = 0; qt < 4 && ready; ++qt) {       // 32 key channels at a time
                     uint32_t sv[32];
@@ -769,7 +775,6 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                         store_state_quarter(ch.hT + (size_t)(32 * qt) * kD + j, srr);
                     }
                 }
-                tmem_ld32(tm + la + COL_O, ov);
                 tmem_wait_ld();
                 if (tid == 0) KDA_TR(TR_S_OLD, c);
                 if (ready) o_step = c;
