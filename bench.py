@@ -369,6 +369,8 @@ def run_gpu(args):
             extra[wl.name] = _measure_workload(wl, dev, stream, args, world, hbm_peak, binding,
                                                inputs)
             torch.cuda.empty_cache()
+        extra["backward_2k"] = _measure_backward(dev, stream, args, world, binding, inputs)
+        torch.cuda.empty_cache()
     decode = None
     if not args.skip_decode:
         decode = _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads)
@@ -410,6 +412,49 @@ def _measure_workload(w, dev, stream, args, world, hbm_peak, binding, inputs):
     return {"tokens": T, "heads": w.H, "sequences": N, "ms": ms,
             "Mtok_s": world * T / (ms * 1e-3) / 1e6, "hbm_gbs": gbs,
             "frac_of_peak": gbs / hbm_peak, "launches_per_step": 1 if not ws_n else 3}
+
+
+# fp32 operations per (token, head) of the backward kernel at d = 128: the
+# checkpoint sweep and the chunk recompute (6 d^2 each: the decayed read and
+# the state update) and the reverse token derivative (18 d^2)
+BWD_FLOPS_PER_TOKEN_HEAD = 30 * 128 * 128
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def _measure_backward(dev, stream, args, world, binding, inputs):
+    """The prefill's gradient (kda_chunk_bwd) on 96 heads x 2,048 tokens, bf16,
+    with dO and dhT given: a correctness-first fp32 CUDA-core kernel, timed
+    for reference."""
+    T, H, d = 2048, 96, 128
+    pre = inputs.make_prefill([T], H, d, d, torch.bfloat16, 1009, 0.02, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(5)
+    dO = torch.randn(T, H, d, generator=gen, device=dev).to(torch.bfloat16)
+    dhT = torch.randn(1, H, d, d, generator=gen, device=dev) * 0.1
+    torch.cuda.synchronize()
+
+    def step():
+        return binding.kda_chunk_bwd(pre.q, pre.k, pre.v, pre.g, pre.beta, dO, pre.h0,
+                                     pre.cu_seqlens, dhT, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    steps = 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    assert binding.kda_stream_status(stream) == binding.KDA_OK
+    ms = _max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    tflops = T * H * BWD_FLOPS_PER_TOKEN_HEAD / (ms * 1e-3) / 1e12
+    return {"tokens": T, "heads": H, "sequences": 1, "ms": ms,
+            "Mtok_s": world * T / (ms * 1e-3) / 1e6, "fp32_tflops": tflops,
+            "frac_of_fp32_peak": tflops / FP32_PEAK_TFLOPS, "launches_per_step": 1}
 
 
 def _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding):
