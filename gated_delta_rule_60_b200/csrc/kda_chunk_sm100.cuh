@@ -1160,14 +1160,17 @@ seg_combine_kernel(const float *__restrict__ M, const float *__restrict__ R,
 // [tokens x 128] x [128 x 128] with the start state as the right factor; it
 // reads and writes each output once and is bound by HBM (about 43 flops per
 // byte), so the warp-level bf16 MMA with fp32 accumulation serves.  CTA: 8
-// warps, 128 tokens a tile (16 per warp), kCorTiles tiles; the start state
-// (transposed, bf16) and the tile sit in shared memory in rows padded to 272
-// bytes, so that each 8 x 8 matrix load touches all banks once.
+// warps, 128 tokens a tile (16 per warp), kCorTiles tiles.  The start state
+// (transposed, bf16) sits in shared memory; each tile's om rows and output
+// rows arrive by asynchronous 16-byte copies into one of two buffers while
+// the previous tile is multiplied, so the loads overlap the math.  Rows are
+// padded to 272 bytes so that each 8 x 8 matrix load touches all banks once.
 constexpr int kCorThreads = 256;
 constexpr int kCorTile = 128;
 constexpr int kCorTiles = 8;
-constexpr int kCorRow = 136;                     // bf16 per padded shared-memory row
-constexpr int kCorSmem = 2 * 128 * kCorRow * 2;  // start state and one tile
+constexpr int kCorRow = 136;                           // bf16 per padded shared-memory row
+constexpr int kCorMat = 128 * kCorRow;                 // elements of one padded 128-row matrix
+constexpr int kCorSmem = 5 * kCorMat * 2;              // start state, 2 x (om tile, o tile)
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -1184,6 +1187,16 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// 16-byte asynchronous copy global -> shared; `bytes` 0 fills the 16 bytes
+// with zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __global__ void __launch_bounds__(kCorThreads)
 seg_correct_kernel(const float *__restrict__ S, const __nv_bfloat16 *__restrict__ om,
                    __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ z,
@@ -1192,34 +1205,52 @@ seg_correct_kernel(const float *__restrict__ S, const __nv_bfloat16 *__restrict_
     if (cu != nullptr && (cu[0] != 0 || (long)cu[1] != T)) return;
     extern __shared__ __align__(16) unsigned char cs_raw[];
     __nv_bfloat16 *sT = reinterpret_cast<__nv_bfloat16 *>(cs_raw);   // [n][k] = S_start[k][n]
-    __nv_bfloat16 *aT = sT + 128 * kCorRow;                          // [token][k] = om
+    __nv_bfloat16 *buf = sT + kCorMat;                               // [2][om tile, o tile]
     const int sg = 1 + (int)blockIdx.z, h = (int)blockIdx.y;
     const long seg_start = seg0_len + (long)(sg - 1) * seg_len;
     const long seg_end = seg_start + seg_len < T ? seg_start + seg_len : T;
     const long t_begin = seg_start + (long)blockIdx.x * (kCorTile * kCorTiles);
     if (t_begin >= seg_end) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    long n_tiles = (seg_end - t_begin + kCorTile - 1) / kCorTile;
+    if (n_tiles > kCorTiles) n_tiles = kCorTiles;
+    // the om and o rows of tile `tile` into buffer `b` (rows past the segment: zeros)
+    auto fetch = [&](int tile, int b) {
+        const long t0 = t_begin + (long)tile * kCorTile;
+        const uint32_t a_s = smem_u32(buf + (size_t)(2 * b) * kCorMat);
+        const uint32_t r_s = smem_u32(buf + (size_t)(2 * b + 1) * kCorMat);
+        for (int c = tid; c < kCorTile * 16; c += kCorThreads) {      // 16-byte chunks, 16 a row
+            const int r = c >> 4, q = c & 15;
+            const bool in = t0 + r < seg_end;
+            const long t = in ? t0 + r : seg_start;                     // a valid address either way
+            const uint32_t off = (uint32_t)(r * kCorRow + 8 * q) * 2u;
+            cp_async16(a_s + off, om + ((size_t)(t - seg0_len) * H + h) * kD + 8 * q, in ? 16u : 0u);
+            cp_async16(r_s + off, o + ((size_t)t * H + h) * kD + 8 * q, in ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    fetch(0, 0);
     const float *Sg = S + ((size_t)sg * H + h) * kD * kD;
     for (int e = tid; e < kD * kD; e += kCorThreads)
         sT[(e & (kD - 1)) * kCorRow + (e >> 7)] = __float2bfloat16_rn(Sg[e]);
     const int g = lane >> 2, tq = lane & 3, rbase = 16 * warp;
-    // this lane's rows of the 8 x 8 matrices: A (tokens x k) and B (n x k)
-    const uint32_t a_addr = smem_u32(aT + (rbase + (lane & 7) + ((lane >> 3) & 1) * 8) * kCorRow +
-                                     (lane >> 4) * 8);
     const uint32_t b_addr = smem_u32(sT + ((lane & 7) + (lane >> 4) * 8) * kCorRow + ((lane >> 3) & 1) * 8);
 #pragma unroll 1
-    for (int tile = 0; tile < kCorTiles; ++tile) {
-        const long t0 = t_begin + (long)tile * kCorTile;
-        if (t0 >= seg_end) break;
-        __syncthreads();              // the start state is written; the last tile's reads are done
-        for (int c = tid; c < kCorTile * 16; c += kCorThreads) {      // 16-byte chunks, 16 a row
-            const int r = c >> 4, q = c & 15;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t0 + r < seg_end)
-                v = *reinterpret_cast<const uint4 *>(om + ((size_t)(t0 + r - seg0_len) * H + h) * kD + 8 * q);
-            *reinterpret_cast<uint4 *>(aT + r * kCorRow + 8 * q) = v;
+    for (int tile = 0; tile < (int)n_tiles; ++tile) {
+        const int b = tile & 1;
+        // the next tile's rows, into the other buffer (freed by the barrier that
+        // closed the previous iteration)
+        if (tile + 1 < (int)n_tiles) {
+            fetch(tile + 1, b ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        __syncthreads();
+        __syncthreads();              // this tile's rows (and the start state) are in place
+        const __nv_bfloat16 *aT = buf + (size_t)(2 * b) * kCorMat;
+        const __nv_bfloat16 *rT = buf + (size_t)(2 * b + 1) * kCorMat;
+        const uint32_t a_addr = smem_u32(aT + (rbase + (lane & 7) + ((lane >> 3) & 1) * 8) * kCorRow +
+                                         (lane >> 4) * 8);
         float acc[16][4];
 #pragma unroll
         for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -1229,22 +1260,24 @@ seg_correct_kernel(const float *__restrict__ S, const __nv_bfloat16 *__restrict_
             ldsm_x4(a, a_addr + kk * 32);
 #pragma unroll
             for (int np = 0; np < 8; ++np) {
-                uint32_t b[4];
-                ldsm_x4(b, b_addr + (np * 16 * kCorRow) * 2 + kk * 32);
-                mma_16816(acc[2 * np], a, b[0], b[1]);
-                mma_16816(acc[2 * np + 1], a, b[2], b[3]);
+                uint32_t bb[4];
+                ldsm_x4(bb, b_addr + (np * 16 * kCorRow) * 2 + kk * 32);
+                mma_16816(acc[2 * np], a, bb[0], bb[1]);
+                mma_16816(acc[2 * np + 1], a, bb[2], bb[3]);
             }
         }
+        const long t0 = t_begin + (long)tile * kCorTile;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            const long t = t0 + rbase + g + 8 * hf;
+            const int r = rbase + g + 8 * hf;
+            const long t = t0 + r;
             if (t >= seg_end) continue;
             __nv_bfloat16 *orow = o + ((size_t)t * H + h) * kD;
             const __nv_bfloat16 *zrow = z ? z + ((size_t)t * H + h) * kD : nullptr;
 #pragma unroll
             for (int nt = 0; nt < 16; ++nt) {
                 const int n = 8 * nt + 2 * tq;
-                const float2 base = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(orow + n));
+                const float2 base = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(rT + r * kCorRow + n));
                 float x0 = base.x + acc[nt][2 * hf], x1 = base.y + acc[nt][2 * hf + 1];
                 if (zrow) {
                     const float2 zz = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(zrow + n));
@@ -1254,6 +1287,7 @@ seg_correct_kernel(const float *__restrict__ S, const __nv_bfloat16 *__restrict_
                 *reinterpret_cast<__nv_bfloat162 *>(orow + n) = __floats2bfloat162_rn(x0, x1);
             }
         }
+        __syncthreads();              // buffer b is free for the tile after next
     }
 }
 
