@@ -40,6 +40,22 @@ struct Smem {
     float red[kThreads / 32];
 };
 
+// Column j of Diag(a) S times k: four independent partial sums, so the FMA
+// latency does not serialise the loop.
+template <int D>
+__device__ __forceinline__ float col_dot_ak(const Smem<D> &sm, int j) {
+    constexpr int R = Smem<D>::kRow;
+    float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < D; i += 4) {
+        r0 = fmaf(sm.a[i] * sm.S[i * R + j], sm.k[i], r0);
+        r1 = fmaf(sm.a[i + 1] * sm.S[(i + 1) * R + j], sm.k[i + 1], r1);
+        r2 = fmaf(sm.a[i + 2] * sm.S[(i + 2) * R + j], sm.k[i + 2], r2);
+        r3 = fmaf(sm.a[i + 3] * sm.S[(i + 3) * R + j], sm.k[i + 3], r3);
+    }
+    return (r0 + r1) + (r2 + r3);
+}
+
 __device__ __forceinline__ float sigmoid_acc(float x) {
     return 1.f / (1.f + expf(-x));
 }
@@ -106,8 +122,7 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
     auto forward_token = [&](float bt) {
         __syncthreads();
         for (int j = tid; j < D; j += kThreads) {      // column j
-            float r = 0.f;
-            for (int i = 0; i < D; ++i) r = fmaf(sm.a[i] * sm.S[i * R + j], sm.k[i], r);
+            const float r = col_dot_ak<D>(sm, j);
             sm.w[j] = sm.v[j] - r;
             sm.u[j] = bt * sm.w[j];
         }
@@ -160,16 +175,20 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             __syncthreads();
             // w = v - S'^T k, u = beta w (S = S_{t-1}, S' = Diag(a) S)
             for (int j = tid; j < D; j += kThreads) {
-                float r = 0.f;
-                for (int i = 0; i < D; ++i) r = fmaf(sm.a[i] * sm.S[i * R + j], sm.k[i], r);
+                const float r = col_dot_ak<D>(sm, j);
                 sm.w[j] = sm.v[j] - r;
                 sm.u[j] = bt * sm.w[j];
             }
             __syncthreads();
             const size_t x = ((size_t)t * H + h) * D;
             // rows: dq = S_t dO = Diag(a) S dO + k (u . dO);  dS += q dO^T;  dk = dS u
-            float udo = 0.f;
-            for (int j = 0; j < D; ++j) udo = fmaf(sm.u[j], sm.dO[j], udo);
+            float udo0 = 0.f, udo1 = 0.f;
+#pragma unroll 4
+            for (int j = 0; j < D; j += 2) {
+                udo0 = fmaf(sm.u[j], sm.dO[j], udo0);
+                udo1 = fmaf(sm.u[j + 1], sm.dO[j + 1], udo1);
+            }
+            const float udo = udo0 + udo1;
             float dk_part[(D + kThreads - 1) / kThreads];
 #pragma unroll
             for (int s = 0; s < (D + kThreads - 1) / kThreads; ++s) dk_part[s] = 0.f;
@@ -177,23 +196,35 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             for (int s = 0; s < (D + kThreads - 1) / kThreads; ++s) {
                 const int i = tid + s * kThreads;
                 if (i >= D) break;
-                float sd = 0.f, dsu = 0.f;
+                float sd0 = 0.f, sd1 = 0.f, dsu0 = 0.f, dsu1 = 0.f;
                 const float qi = sm.q[i];
-                for (int j = 0; j < D; ++j) {
-                    sd = fmaf(sm.S[i * R + j], sm.dO[j], sd);
-                    const float ds = fmaf(qi, sm.dO[j], sm.dS[i * R + j]);
-                    sm.dS[i * R + j] = ds;
-                    dsu = fmaf(ds, sm.u[j], dsu);
+#pragma unroll 4
+                for (int j = 0; j < D; j += 2) {
+                    sd0 = fmaf(sm.S[i * R + j], sm.dO[j], sd0);
+                    sd1 = fmaf(sm.S[i * R + j + 1], sm.dO[j + 1], sd1);
+                    const float ds0 = fmaf(qi, sm.dO[j], sm.dS[i * R + j]);
+                    const float ds1 = fmaf(qi, sm.dO[j + 1], sm.dS[i * R + j + 1]);
+                    sm.dS[i * R + j] = ds0;
+                    sm.dS[i * R + j + 1] = ds1;
+                    dsu0 = fmaf(ds0, sm.u[j], dsu0);
+                    dsu1 = fmaf(ds1, sm.u[j + 1], dsu1);
                 }
-                IO<T>::st(dq + x + i, fmaf(sm.a[i], sd, sm.k[i] * udo));
-                dk_part[s] = dsu;
+                IO<T>::st(dq + x + i, fmaf(sm.a[i], sd0 + sd1, sm.k[i] * udo));
+                dk_part[s] = dsu0 + dsu1;
             }
             __syncthreads();
             // columns: du = dS^T k;  dv = beta du
             float dbp = 0.f;
             for (int j = tid; j < D; j += kThreads) {
-                float d = 0.f;
-                for (int i = 0; i < D; ++i) d = fmaf(sm.dS[i * R + j], sm.k[i], d);
+                float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll 4
+                for (int i = 0; i < D; i += 4) {
+                    d0 = fmaf(sm.dS[i * R + j], sm.k[i], d0);
+                    d1 = fmaf(sm.dS[(i + 1) * R + j], sm.k[i + 1], d1);
+                    d2 = fmaf(sm.dS[(i + 2) * R + j], sm.k[i + 2], d2);
+                    d3 = fmaf(sm.dS[(i + 3) * R + j], sm.k[i + 3], d3);
+                }
+                const float d = (d0 + d1) + (d2 + d3);
                 sm.du[j] = d;
                 IO<T>::st(dv + x + j, bt * d);
                 dbp = fmaf(d, sm.w[j], dbp);
@@ -206,16 +237,21 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
                 const int i = tid + s * kThreads;
                 if (i >= D) break;
                 const float ai = sm.a[i], bki = bt * sm.k[i];
-                float sdu = 0.f, da = 0.f;
-                for (int j = 0; j < D; ++j) {
-                    const float sij = sm.S[i * R + j];
-                    sdu = fmaf(sij, sm.du[j], sdu);
-                    const float dsp = fmaf(-bki, sm.du[j], sm.dS[i * R + j]);
-                    da = fmaf(dsp, sij, da);
-                    sm.dS[i * R + j] = ai * dsp;
+                float sdu0 = 0.f, sdu1 = 0.f, da0 = 0.f, da1 = 0.f;
+#pragma unroll 4
+                for (int j = 0; j < D; j += 2) {
+                    const float s0 = sm.S[i * R + j], s1 = sm.S[i * R + j + 1];
+                    sdu0 = fmaf(s0, sm.du[j], sdu0);
+                    sdu1 = fmaf(s1, sm.du[j + 1], sdu1);
+                    const float p0 = fmaf(-bki, sm.du[j], sm.dS[i * R + j]);
+                    const float p1 = fmaf(-bki, sm.du[j + 1], sm.dS[i * R + j + 1]);
+                    da0 = fmaf(p0, s0, da0);
+                    da1 = fmaf(p1, s1, da1);
+                    sm.dS[i * R + j] = ai * p0;
+                    sm.dS[i * R + j + 1] = ai * p1;
                 }
-                IO<T>::st(dk + x + i, dk_part[s] - bt * ai * sdu);
-                IO<T>::st(dg + x + i, da * ai * sm.lg[i]);
+                IO<T>::st(dk + x + i, dk_part[s] - bt * ai * (sdu0 + sdu1));
+                IO<T>::st(dg + x + i, (da0 + da1) * ai * sm.lg[i]);
             }
             // dbeta = du . w (block reduction)
             for (int o = 16; o > 0; o >>= 1) dbp += __shfl_xor_sync(0xffffffffu, dbp, o);
