@@ -90,6 +90,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                  ctypes.c_int, vp, vp, vp, vp, vp]
     lib.kda_debug_stall_prefill.restype = ctypes.c_int
     lib.kda_debug_stall_prefill.argtypes = [i32, ctypes.c_uint64]
+    lib.kda_debug_range_prefill.restype = ctypes.c_int
+    lib.kda_debug_range_prefill.argtypes = [i32]
+    lib.kda_debug_range_read.restype = ctypes.c_int
+    lib.kda_debug_range_read.argtypes = [ctypes.POINTER(ctypes.c_float), sz]
     _lib = lib
     return lib
 
@@ -445,6 +449,30 @@ def kda_debug_stall_prefill(step: int, limit_cycles: int) -> None:
     st = load_library().kda_debug_stall_prefill(int(step), int(limit_cycles))
     if st != KDA_OK:
         raise KdaError(st, "kda_debug_stall_prefill")
+
+
+RANGE_ROWS = ("Kr", "Qr", "Kh", "Z")
+RANGE_COLS = ("max_abs", "min_nonzero_abs", "subnormal", "zero", "nonfinite", "count")
+
+
+def kda_debug_range_prefill(step: int) -> None:
+    """Make CTA 0 of the next tensor-core kda_chunk_fwd call record the
+    magnitudes of its scaled operands (Kr, Qr, Kh in bf16) and of Z = Kh^T T
+    (fp32, before the delta rescale) at state step `step`."""
+    st = load_library().kda_debug_range_prefill(int(step))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_debug_range_prefill")
+
+
+def kda_debug_range_read() -> dict:
+    """The record of kda_debug_range_prefill: {row: {column: value}}."""
+    buf = (ctypes.c_float * (len(RANGE_ROWS) * len(RANGE_COLS)))()
+    st = load_library().kda_debug_range_read(buf, len(buf))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_debug_range_read")
+    n = len(RANGE_COLS)
+    return {r: {c: float(buf[i * n + j]) for j, c in enumerate(RANGE_COLS)}
+            for i, r in enumerate(RANGE_ROWS)}
 
 
 def kda_stream_status(stream=None) -> int:

@@ -3,6 +3,7 @@
 // One translation unit holds every kernel so that the per-device status word
 // (kda_common.cuh) is a single symbol.  See include/kda.h for the contract of
 // each entry point.
+#include <cstring>
 #include "../../include/kda.h"
 
 #include "kda_common.cuh"
@@ -386,6 +387,32 @@ kda_status kda_debug_stall_prefill(int32_t step, uint64_t limit_cycles) {
     kda::DebugStall &d = kda::debug_stall();
     d.limit.store((unsigned long long)limit_cycles);
     d.step.store(step);
+    return KDA_OK;
+}
+
+kda_status kda_debug_range_prefill(int32_t step) {
+    if (step < 0) return KDA_ERR_INVALID_ARGUMENT;
+    static const unsigned int init[4][kda::prefill::kRangeCols] = {
+        {0u, 0x7f800000u, 0u, 0u, 0u, 0u}, {0u, 0x7f800000u, 0u, 0u, 0u, 0u},
+        {0u, 0x7f800000u, 0u, 0u, 0u, 0u}, {0u, 0x7f800000u, 0u, 0u, 0u, 0u}};
+    if (cudaMemcpyToSymbol(kda::prefill::g_range, init, sizeof(init)) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kda::debug_range().step.store(step);
+    return KDA_OK;
+}
+
+kda_status kda_debug_range_read(float *out, size_t n) {
+    unsigned int r[4][kda::prefill::kRangeCols];
+    if (out == nullptr || n < 4 * (size_t)kda::prefill::kRangeCols) return KDA_ERR_INVALID_ARGUMENT;
+    if (cudaMemcpyFromSymbol(r, kda::prefill::g_range, sizeof(r)) != cudaSuccess) return KDA_ERR_CUDA;
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < kda::prefill::kRangeCols; ++j) {
+            uint32_t b = r[i][j];
+            float f;
+            if (j <= kda::prefill::kRangeMinNz) std::memcpy(&f, &b, 4);
+            else f = (float)b;
+            out[i * kda::prefill::kRangeCols + j] = f;
+        }
     return KDA_OK;
 }
 

@@ -184,6 +184,7 @@ struct Params {
     float *ws_R, *ws_M, *ws_S;    // [G][H][128][128] each (segment modes)
     unsigned long long wait_limit;  // bound of a pipeline wait, SM clock cycles
     int stall_step;               // diagnostic: step at which the scan waits on `never` (-1: none)
+    int range_step;               // diagnostic: step whose operands CTA 0 records (-1: none)
 };
 
 // What one CTA runs: a token range of one head, where its state starts and
@@ -340,6 +341,74 @@ __device__ __forceinline__ void fail(Barriers &bars) {
     raise_error(kErrTimeout);
 }
 
+// 32 values of one lane, passed by value to the out-of-line helpers below.
+struct OutRegs {
+    uint32_t v[kStep];
+};
+
+// Diagnostic range record (test-only): magnitudes of one step's scaled
+// operands as the kernel forms them.  Rows: Kr, Qr, Kh (bf16, written by the
+// gate pass) and Z = Kh^T T (fp32, read from tensor memory before the delta
+// rescale).  Columns: max |x| and min nonzero |x| (float bits), then counts of
+// subnormals, zeros, non-finite values and all values.
+enum { kRangeMax = 0, kRangeMinNz, kRangeSub, kRangeZero, kRangeNonFinite, kRangeCount, kRangeCols };
+__device__ unsigned int g_range[4][kRangeCols];
+
+__device__ __forceinline__ void range_add(int row, float m, float mn, unsigned sub, unsigned zero,
+                                          unsigned nonfin, unsigned cnt) {
+    atomicMax(&g_range[row][kRangeMax], __float_as_uint(m));
+    atomicMin(&g_range[row][kRangeMinNz], __float_as_uint(mn));
+    atomicAdd(&g_range[row][kRangeSub], sub);
+    atomicAdd(&g_range[row][kRangeZero], zero);
+    atomicAdd(&g_range[row][kRangeNonFinite], nonfin);
+    atomicAdd(&g_range[row][kRangeCount], cnt);
+}
+
+// The bf16 operands of the tile slot, after the gate pass (one prep warpgroup).
+__device__ __noinline__ void range_probe_operands(const unsigned char *slot, int pt) {
+    const uint32_t base[3][2] = {{SL_K0, SL_K1}, {SL_Q0, SL_Q1}, {SL_G0, SL_G1}};
+#pragma unroll 1
+    for (int row = 0; row < 3; ++row) {
+        float m = 0.f, mn = __uint_as_float(0x7f800000u);
+        unsigned sub = 0, zero = 0, nonfin = 0, cnt = 0;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            const uint16_t *e = reinterpret_cast<const uint16_t *>(slot + base[row][half]);
+#pragma unroll 1
+            for (int i = pt; i < kStep * 64; i += 128) {
+                const uint16_t b = e[i];
+                const uint16_t ex = (b >> 7) & 0xff, man = b & 0x7f;
+                const float a = fabsf(__uint_as_float((uint32_t)b << 16));
+                ++cnt;
+                if (ex == 0xff) { ++nonfin; continue; }
+                if (ex == 0 && man == 0) { ++zero; continue; }
+                if (ex == 0) ++sub;
+                m = fmaxf(m, a);
+                mn = fminf(mn, a);
+            }
+        }
+        range_add(row, m, mn, sub, zero, nonfin, cnt);
+    }
+}
+
+// Z = Kh^T T for this thread's key channel, 32 columns, before the delta rescale.
+__device__ __noinline__ void range_probe_z(OutRegs zv) {
+    float m = 0.f, mn = __uint_as_float(0x7f800000u);
+    unsigned sub = 0, zero = 0, nonfin = 0;
+#pragma unroll 1
+    for (int c = 0; c < kStep; ++c) {
+        const uint32_t b = zv.v[c];
+        const uint32_t ex = (b >> 23) & 0xff, man = b & 0x7fffff;
+        const float a = fabsf(__uint_as_float(b));
+        if (ex == 0xff) { ++nonfin; continue; }
+        if (ex == 0 && man == 0) { ++zero; continue; }
+        if (ex == 0) ++sub;
+        m = fmaxf(m, a);
+        mn = fminf(mn, a);
+    }
+    range_add(3, m, mn, sub, zero, nonfin, kStep);
+}
+
 // Diagnostic stall (out of line, off the steady-state instruction stream).
 __device__ __noinline__ void stall_here(Barriers &bars, volatile int *abort, unsigned long long limit) {
     if (!warp_wait(&bars.never, 0, abort, limit)) fail(bars);
@@ -431,9 +500,6 @@ __device__ __noinline__ void gate_pass_partial(unsigned char *slot, int pw, int 
 }
 
 // Masked plain stores of the last, partial step's outputs (out of line).
-struct OutRegs {
-    uint32_t v[kStep];
-};
 __device__ __noinline__ void store_o_partial(__nv_bfloat16 *dst, size_t step, int Lc, OutRegs ov) {
 #pragma unroll 1
     for (int r = 0; r < Lc; ++r) dst[(size_t)r * step] = __float2bfloat16_rn(__uint_as_float(ov.v[r]));
@@ -447,7 +513,9 @@ __device__ __noinline__ void store_state_quarter(float *dst, OutRegs sv) {
 
 // kGate: the fused output gate o * sigmoid(z) (p.z), compiled only into the
 // gated instantiation so that the plain operator carries no trace of it.
-template <bool kGate>
+// kProbe: the diagnostic range record, compiled only into the instantiation
+// a kda_debug_range_prefill call launches.
+template <bool kGate, bool kProbe = false>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
@@ -858,6 +926,7 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             fence_proxy_async_smem();
             group_sync(bar_id);                                             // operands written
+            if (kProbe && s == p.range_step && blockIdx.x == 0) range_probe_operands(slot, pt);
 
             // ---------------- A_kk (TMEM lanes 0-31) and A_qk (lanes 32-63)
             if (iss && !*abortp) {
@@ -1052,6 +1121,12 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 uint32_t zv[32];
                 tmem_ld32(tPl, zv);
                 tmem_wait_ld();
+                if (kProbe && s == p.range_step && blockIdx.x == 0) {
+                    OutRegs zr;
+#pragma unroll
+                    for (int c2 = 0; c2 < kStep; ++c2) zr.v[c2] = zv[c2];
+                    range_probe_z(zr);
+                }
                 const int i = 32 * pw + lane;           // key channel
                 const float di = dlt[i];
 #pragma unroll
@@ -1397,6 +1472,14 @@ inline SegPlan plan_segments(int N, int64_t T, int H) {
 // One-shot diagnostic (kda_debug_stall_prefill): the next tensor-core
 // prefill call makes every CTA's scan wait, at step `step`, on a barrier that
 // nothing arrives on, with a bound of `limit` cycles.
+struct DebugRange {
+    std::atomic<int> step{-1};
+};
+inline DebugRange &debug_range() {
+    static DebugRange d;
+    return d;
+}
+
 struct DebugStall {
     std::atomic<int> step{-1};
     std::atomic<unsigned long long> limit{0};
@@ -1429,7 +1512,10 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
         !make_qkvg_map(&mv, base(v), H, T_map) || !make_qkvg_map(&mg, base(g), H, T_map) ||
         !make_qkvg_map(&mo, base(o), H, T_map))
         return KDA_ERR_CUDA;
-    auto kern = z ? prefill::chunk_fwd_sm100_kernel<true> : prefill::chunk_fwd_sm100_kernel<false>;
+    const int range_step = debug_range().step.exchange(-1);
+    auto kern = z ? prefill::chunk_fwd_sm100_kernel<true>
+                  : (range_step >= 0 ? prefill::chunk_fwd_sm100_kernel<false, true>
+                                     : prefill::chunk_fwd_sm100_kernel<false>);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)prefill::kSmemAlloc) != cudaSuccess)
         return KDA_ERR_CUDA;
@@ -1450,6 +1536,7 @@ inline kda_status sm100_chunk_fwd(const void *q, const void *k, const void *v, c
     p.ws_R = p.ws_M = p.ws_S = nullptr;
     p.om = nullptr;
     p.stall_step = debug_stall().step.exchange(-1);
+    p.range_step = range_step;
     const unsigned long long lim = debug_stall().limit.exchange(0);
     p.wait_limit = (p.stall_step >= 0 && lim > 0) ? lim : prefill::kWaitLimit;
     const SegPlan pl = plan_segments(N, T_tot, H);

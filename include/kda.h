@@ -316,6 +316,27 @@ KDA_API kda_status kda_selftest_wait_timeout(uint64_t limit_cycles, void *stream
  */
 KDA_API kda_status kda_debug_stall_prefill(int32_t step, uint64_t limit_cycles);
 
+/*
+ * Diagnostic (test-only) record of the magnitudes the tensor-core prefill
+ * forms inside one step, the evidence for the bf16 range claim of the bounded
+ * gate (page "Kimi K3 发布核实与 Moonshot AI 主干架构演变", §3 "K3 对 Kimi
+ * Linear 的进一步修改", bullet 1: reciprocal decay scaling inside a 16-token
+ * tile stays within the BF16 range).  kda_debug_range_prefill(step) clears the
+ * record and makes CTA 0 (the first (sequence, head) chain) of the NEXT
+ * tensor-core kda_chunk_fwd call record its operands at state step `step`
+ * (32 tokens): the scaled keys Kr = K e^{b-m}, queries Qr = Q e^{b-m} and
+ * keys Kh = K e^{m-b} as the gate pass writes them (bf16), and Z = Kh^T T
+ * before the delta rescale (fp32, from tensor memory).  The setting is
+ * consumed by that one call.  Returns KDA_ERR_INVALID_ARGUMENT for step < 0.
+ *
+ * kda_debug_range_read(out, n) copies the record, n >= 24 floats, row by row
+ * for Kr, Qr, Kh, Z: max |x|, min nonzero |x|, then the counts of subnormal,
+ * zero, non-finite and all values (as floats).  Call it after the prefill
+ * completed (e.g. after kda_stream_status).
+ */
+KDA_API kda_status kda_debug_range_prefill(int32_t step);
+KDA_API kda_status kda_debug_range_read(float *out, size_t n);
+
 /* Static English description of a status code (never NULL). */
 KDA_API const char *kda_status_string(kda_status s);
 

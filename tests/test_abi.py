@@ -174,6 +174,10 @@ def test_selftest_limit_is_checked_on_the_host(lib):
 
 def test_prefill_stall_diagnostic_checks_its_arguments(lib):
     """Invalid requests are refused on the host and arm nothing."""
+    assert lib.kda_debug_range_prefill(-1) == binding.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_debug_range_read(None, 24) == binding.KDA_ERR_INVALID_ARGUMENT
+    buf = (ctypes.c_float * 8)()
+    assert lib.kda_debug_range_read(buf, 8) == binding.KDA_ERR_INVALID_ARGUMENT
     assert lib.kda_debug_stall_prefill(-1, 1000) == binding.KDA_ERR_INVALID_ARGUMENT
     assert lib.kda_debug_stall_prefill(0, 0) == binding.KDA_ERR_INVALID_ARGUMENT
     assert lib.kda_debug_stall_prefill(0, (1 << 32) + 1) == binding.KDA_ERR_INVALID_ARGUMENT
