@@ -56,6 +56,48 @@ __device__ __forceinline__ float col_dot_ak(const Smem<D> &sm, int j) {
     return (r0 + r1) + (r2 + r3);
 }
 
+// Copies between a padded shared-memory matrix (rows of D + 1 floats) and a
+// dense D x D global array, 16 bytes per global access, eight accesses in
+// flight per thread (the reverse sweep moves one 64 KB state per token).
+template <int D>
+__device__ __forceinline__ void mat_from_global(float *sdst, const float *__restrict__ src, int tid) {
+    constexpr int R = D + 1, N4 = D * D / 4, B = 8;
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll 1
+    for (int base = tid; base < N4; base += B * kThreads) {
+        float4 v[B];
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int e4 = base + u * kThreads;
+            v[u] = e4 < N4 ? s4[e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            const int e4 = base + u * kThreads;
+            if (e4 < N4) {
+                const int e = 4 * e4, i = e / D, j = e % D;
+                float *d = sdst + i * R + j;
+                d[0] = v[u].x;
+                d[1] = v[u].y;
+                d[2] = v[u].z;
+                d[3] = v[u].w;
+            }
+        }
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void mat_to_global(float *__restrict__ dst, const float *ssrc, int tid) {
+    constexpr int R = D + 1, N4 = D * D / 4;
+    float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll 4
+    for (int e4 = tid; e4 < N4; e4 += kThreads) {
+        const int e = 4 * e4, i = e / D, j = e % D;
+        const float *sp = ssrc + i * R + j;
+        d4[e4] = make_float4(sp[0], sp[1], sp[2], sp[3]);
+    }
+}
+
 __device__ __forceinline__ float sigmoid_acc(float x) {
     return 1.f / (1.f + expf(-x));
 }
@@ -135,13 +177,16 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
     auto beta_of = [&](int64_t t) { return IO<T>::ld(beta + (size_t)t * H + h); };
 
     // ---- forward sweep: checkpoints before every 16th token
-    for (int e = tid; e < D * D; e += kThreads)
-        sm.S[(e / D) * R + e % D] = h0 ? h0[unit * DD + e] : 0.f;
+    if (h0) {
+        mat_from_global<D>(sm.S, h0 + unit * DD, tid);
+    } else {
+        for (int e = tid; e < D * D; e += kThreads) sm.S[(e / D) * R + e % D] = 0.f;
+    }
     for (int64_t t = s0; t < s1; ++t) {
         if ((t - s0) % kChunk == 0) {
             __syncthreads();
             float *dst = ck + (size_t)((t - s0) / kChunk) * DD;
-            for (int e = tid; e < D * D; e += kThreads) dst[e] = sm.S[(e / D) * R + e % D];
+            mat_to_global<D>(dst, sm.S, tid);
         }
         __syncthreads();
         load_token(t, false);
@@ -150,26 +195,28 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
 
     // ---- reverse sweep
     __syncthreads();
-    for (int e = tid; e < D * D; e += kThreads)
-        sm.dS[(e / D) * R + e % D] = dhT ? dhT[unit * DD + e] : 0.f;
+    if (dhT) {
+        mat_from_global<D>(sm.dS, dhT + unit * DD, tid);
+    } else {
+        for (int e = tid; e < D * D; e += kThreads) sm.dS[(e / D) * R + e % D] = 0.f;
+    }
     for (int64_t c = n_chunks(L) - 1; c >= 0; --c) {
         const int64_t a0 = s0 + c * kChunk;
         const int64_t a1 = a0 + kChunk < s1 ? a0 + kChunk : s1;
         // the chunk's token states S_{t-1}, recomputed from its checkpoint
         __syncthreads();
-        for (int e = tid; e < D * D; e += kThreads)
-            sm.S[(e / D) * R + e % D] = ck[(size_t)c * DD + e];
+        mat_from_global<D>(sm.S, ck + (size_t)c * DD, tid);
         for (int64_t t = a0; t < a1; ++t) {
             __syncthreads();
             float *dst = tk + (size_t)(t - a0) * DD;
-            for (int e = tid; e < D * D; e += kThreads) dst[e] = sm.S[(e / D) * R + e % D];
+            mat_to_global<D>(dst, sm.S, tid);
             load_token(t, false);
             forward_token(beta_of(t));
         }
         for (int64_t t = a1 - 1; t >= a0; --t) {
             __syncthreads();
             const float *src = tk + (size_t)(t - a0) * DD;
-            for (int e = tid; e < D * D; e += kThreads) sm.S[(e / D) * R + e % D] = src[e];
+            mat_from_global<D>(sm.S, src, tid);
             load_token(t, true);
             const float bt = beta_of(t);
             __syncthreads();
@@ -266,7 +313,7 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
     }
     __syncthreads();
     if (dh0)
-        for (int e = tid; e < D * D; e += kThreads) dh0[unit * DD + e] = sm.dS[(e / D) * R + e % D];
+        mat_to_global<D>(dh0 + unit * DD, sm.dS, tid);
 }
 
 }  // namespace bwd
