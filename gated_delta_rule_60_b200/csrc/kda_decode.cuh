@@ -131,6 +131,7 @@ decode_step_d128_kernel(const T *__restrict__ q, const T *__restrict__ k,
     constexpr int D = 128, W = kDecode128Threads / 32, R = D / W;
     __shared__ float sa[D], sk[D], sq[D], su[D];
     __shared__ float4 sr[W][D / 4], sp[W][D / 4];
+    __shared__ float skq[W];
     const long u = blockIdx.x;
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     float *Su = S + (size_t)u * D * D + (size_t)(R * w) * D + 4 * l;
@@ -158,12 +159,18 @@ decode_step_d128_kernel(const T *__restrict__ q, const T *__restrict__ k,
     }
     sr[w][l] = r;
     sp[w][l] = p;
+    if (l == 0) {                                   // k . q over this warp's rows
+        float kq = 0.f;
+#pragma unroll
+        for (int i = 0; i < R; ++i) kq = fmaf(sk[R * w + i], sq[R * w + i], kq);
+        skq[w] = kq;
+    }
     __syncthreads();
     if (tid < D) {
         const int j = tid;
         float kq = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; ++i) kq = fmaf(sk[i], sq[i], kq);
+#pragma unroll
+        for (int x = 0; x < W; ++x) kq += skq[x];
         const float *srf = reinterpret_cast<const float *>(sr);
         const float *spf = reinterpret_cast<const float *>(sp);
         float rj = 0.f, pj = 0.f;
