@@ -102,7 +102,7 @@ kda_status launch_bwd(const void *q, const void *k, const void *v, const void *g
     const size_t DD = (size_t)D * D;
     float *ckpt = static_cast<float *>(ws);
     float *tok = ckpt + (size_t)H * ((T_tot + kda::bwd::kChunk - 1) / kda::bwd::kChunk + N) * DD;
-    kern<<<(unsigned)(N * H), kda::bwd::kThreads, smem, s>>>(
+    kern<<<(unsigned)(N * H), kda::bwd::threads_of<D>(), smem, s>>>(
         (const T *)q, (const T *)k, (const T *)v, (const T *)g, (const T *)beta, h0, cu, N, T_tot,
         H, (const T *)dO, dhT, (T *)dq, (T *)dk, (T *)dv, (T *)dg, (T *)dbeta, dh0, ckpt, tok);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
