@@ -140,22 +140,48 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
     float *ck = ckpt + ((size_t)base * H + (size_t)h * n_chunks(L)) * DD;
     float *tk = tok + unit * kChunk * DD;
 
-    auto load_vec = [&](float *dst, const T *src) {
-        for (int i = tid; i < D; i += NT) dst[i] = IO<T>::ld(src + i);
-    };
-    // token t's inputs into shared memory (a = decay, lg = dl/dg)
-    auto load_token = [&](int64_t t, bool grads) {
-        const size_t x = ((size_t)t * H + h) * D;
-        load_vec(sm.q, q + x);
-        load_vec(sm.k, k + x);
-        load_vec(sm.v, v + x);
-        for (int i = tid; i < D; i += NT) {
-            const float gi = IO<T>::ld(g + x + i);
-            const float s = sigmoid_acc(gi);
-            sm.a[i] = expf(-5.f * s);
-            sm.lg[i] = -5.f * s * (1.f - s);
+    // token t's inputs: fetched into registers (thread i < D holds element i
+    // of each vector, every thread holds beta) and written to shared memory
+    // one token later, so that the loads fly while the previous token runs
+    struct TokIn { float q, k, v, g, dO, beta; };
+    auto fetch_token = [&](int64_t t, bool grads) {
+        TokIn r{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const size_t x = ((size_t)t * H + h) * D + tid;
+        if (tid < D) {
+            r.q = IO<T>::ld(q + x);
+            r.k = IO<T>::ld(k + x);
+            r.v = IO<T>::ld(v + x);
+            r.g = IO<T>::ld(g + x);
+            if (grads) r.dO = IO<T>::ld(dO + x);
         }
-        if (grads) load_vec(sm.dO, dO + x);
+        r.beta = IO<T>::ld(beta + (size_t)t * H + h);
+        return r;
+    };
+    // a = decay, lg = dl/dg
+    auto put_token = [&](const TokIn &r) {
+        if (tid < D) {
+            const float s = sigmoid_acc(r.g);
+            sm.q[tid] = r.q;
+            sm.k[tid] = r.k;
+            sm.v[tid] = r.v;
+            sm.a[tid] = expf(-5.f * s);
+            sm.lg[tid] = -5.f * s * (1.f - s);
+            sm.dO[tid] = r.dO;
+        }
+    };
+    // one token state (D x D fp32) through registers, 16 bytes per access
+    constexpr int kPf = D / 16;                      // float4 per thread
+    auto fetch_state = [&](float4 (&pf)[kPf], const float *src) {
+        const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+        for (int u = 0; u < kPf; ++u) pf[u] = s4[tid + u * NT];
+    };
+    auto put_state = [&](const float4 (&pf)[kPf]) {
+#pragma unroll
+        for (int u = 0; u < kPf; ++u) {
+            const int e = 4 * (tid + u * NT);
+            *reinterpret_cast<float4 *>(sm.S + (e / D) * R + e % D) = pf[u];
+        }
     };
     // column idx of Diag(a) S times k (rows part, part + 4, ...)
     auto col_ak = [&]() {
@@ -190,19 +216,22 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             }
         }
     };
-    auto beta_of = [&](int64_t t) { return IO<T>::ld(beta + (size_t)t * H + h); };
 
     // ---- forward sweep: checkpoints before every 16th token
     if (h0) mat_from_global<D>(sm.S, h0 + unit * DD, tid);
     else mat_zero<D>(sm.S, tid);
+    TokIn ti{0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (s0 < s1) ti = fetch_token(s0, false);
     for (int64_t t = s0; t < s1; ++t) {
         if ((t - s0) % kChunk == 0) {
             __syncthreads();
             mat_to_global<D>(ck + (size_t)((t - s0) / kChunk) * DD, sm.S, tid);
         }
         __syncthreads();
-        load_token(t, false);
-        forward_token(beta_of(t));
+        put_token(ti);
+        const float bt = ti.beta;
+        if (t + 1 < s1) ti = fetch_token(t + 1, false);
+        forward_token(bt);
     }
 
     // ---- reverse sweep
@@ -215,17 +244,30 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         // the chunk's token states S_{t-1}, recomputed from its checkpoint
         __syncthreads();
         mat_from_global<D>(sm.S, ck + (size_t)c * DD, tid);
+        ti = fetch_token(a0, false);
         for (int64_t t = a0; t < a1; ++t) {
             __syncthreads();
             mat_to_global<D>(tk + (size_t)(t - a0) * DD, sm.S, tid);
-            load_token(t, false);
-            forward_token(beta_of(t));
+            put_token(ti);
+            const float bt = ti.beta;
+            if (t + 1 < a1) ti = fetch_token(t + 1, false);
+            forward_token(bt);
         }
+        // the reverse pass over the chunk: token t - 1's state and inputs load
+        // while token t is differentiated
+        __syncthreads();
+        float4 pf[kPf];
+        fetch_state(pf, tk + (size_t)(a1 - 1 - a0) * DD);
+        ti = fetch_token(a1 - 1, true);
         for (int64_t t = a1 - 1; t >= a0; --t) {
             __syncthreads();
-            mat_from_global<D>(sm.S, tk + (size_t)(t - a0) * DD, tid);
-            load_token(t, true);
-            const float bt = beta_of(t);
+            put_state(pf);
+            put_token(ti);
+            const float bt = ti.beta;
+            if (t > a0) {
+                fetch_state(pf, tk + (size_t)(t - 1 - a0) * DD);
+                ti = fetch_token(t - 1, true);
+            }
             __syncthreads();
             // w = v - S'^T k, u = beta w (S = S_{t-1}, S' = Diag(a) S)
             {
