@@ -21,7 +21,10 @@
 // of the current pass, each a quarter of it (every fourth element), and meet
 // in two shuffles; the CTA has 4 d threads.  State rows are padded to d + 8
 // floats in shared memory, so that a column pass reads 32 distinct banks per
-// warp and a row pass at most two-way conflicting ones.
+// warp and a row pass at most two-way conflicting ones.  A reverse token takes
+// two passes: one over columns, for S'^T k and du, using
+// du = (dS + q dO^T)^T k = dS^T k + dO (q . k) on dS as it enters, and one over
+// rows for everything else.
 #pragma once
 
 #include "kda_common.cuh"
@@ -40,8 +43,10 @@ struct Smem {
     static constexpr int kRow = D + 8;               // padded row stride
     float S[D * kRow];
     float dS[D * kRow];
+    static constexpr int kQkParts = D >= 32 ? D / 32 : 1;   // warps holding q and k
     float q[D], k[D], v[D], a[D], lg[D], dO[D], u[D], w[D], du[D];
     float red[threads_of<D>() / 32];
+    float qkp[kQkParts];                             // per-warp partial sums of q . k
 };
 
 // Sum over the four lanes of a row or column.
@@ -157,8 +162,14 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         r.beta = IO<T>::ld(beta + (size_t)t * H + h);
         return r;
     };
-    // a = decay, lg = dl/dg
-    auto put_token = [&](const TokIn &r) {
+    // a = decay, lg = dl/dg; with grads, also the partial sums of q . k
+    auto put_token = [&](const TokIn &r, bool grads) {
+        if (grads && tid < 32 * Smem<D>::kQkParts) {
+            float p = tid < D ? r.q * r.k : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            if ((tid & 31) == 0) sm.qkp[tid >> 5] = p;
+        }
         if (tid < D) {
             const float s = sigmoid_acc(r.g);
             sm.q[tid] = r.q;
@@ -228,7 +239,7 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             mat_to_global<D>(ck + (size_t)((t - s0) / kChunk) * DD, sm.S, tid);
         }
         __syncthreads();
-        put_token(ti);
+        put_token(ti, false);
         const float bt = ti.beta;
         if (t + 1 < s1) ti = fetch_token(t + 1, false);
         forward_token(bt);
@@ -248,7 +259,7 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         for (int64_t t = a0; t < a1; ++t) {
             __syncthreads();
             mat_to_global<D>(tk + (size_t)(t - a0) * DD, sm.S, tid);
-            put_token(ti);
+            put_token(ti, false);
             const float bt = ti.beta;
             if (t + 1 < a1) ti = fetch_token(t + 1, false);
             forward_token(bt);
@@ -262,24 +273,45 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         for (int64_t t = a1 - 1; t >= a0; --t) {
             __syncthreads();
             put_state(pf);
-            put_token(ti);
+            put_token(ti, true);
             const float bt = ti.beta;
             if (t > a0) {
                 fetch_state(pf, tk + (size_t)(t - 1 - a0) * DD);
                 ti = fetch_token(t - 1, true);
             }
             __syncthreads();
-            // w = v - S'^T k, u = beta w (S = S_{t-1}, S' = Diag(a) S)
+            const size_t x = ((size_t)t * H + h) * D;
+            // columns: w = v - S'^T k, u = beta w (S = S_{t-1}, S' = Diag(a) S);
+            // du = (dS + q dO^T)^T k = dS^T k + dO (q . k);  dv = beta du
+            float dbp = 0.f;
             {
-                const float r = col_ak();
+                const int j = idx;
+                float r0 = 0.f, r1 = 0.f, d0 = 0.f, d1 = 0.f;
+#pragma unroll 4
+                for (int s = 0; s < Q; s += 2) {
+                    const int i0 = kParts * s + part, i1 = i0 + kParts;
+                    const float k0 = sm.k[i0], k1 = sm.k[i1];
+                    r0 = fmaf(sm.a[i0] * sm.S[i0 * R + j], k0, r0);
+                    r1 = fmaf(sm.a[i1] * sm.S[i1 * R + j], k1, r1);
+                    d0 = fmaf(sm.dS[i0 * R + j], k0, d0);
+                    d1 = fmaf(sm.dS[i1 * R + j], k1, d1);
+                }
+                const float r = quad_sum(r0 + r1), dsk = quad_sum(d0 + d1);
                 if (part == 0) {
-                    sm.w[idx] = sm.v[idx] - r;
-                    sm.u[idx] = bt * sm.w[idx];
+                    float qk = 0.f;
+#pragma unroll
+                    for (int p = 0; p < Smem<D>::kQkParts; ++p) qk += sm.qkp[p];
+                    const float wj = sm.v[j] - r, du = fmaf(sm.dO[j], qk, dsk);
+                    sm.u[j] = bt * wj;
+                    sm.du[j] = du;
+                    IO<T>::st(dv + x + j, bt * du);
+                    dbp = du * wj;
                 }
             }
             __syncthreads();
-            const size_t x = ((size_t)t * H + h) * D;
-            // rows: dq = S_t dO = Diag(a) S dO + k (u . dO);  dS += q dO^T;  dk = dS u
+            // rows, one pass: dq = S_t dO = Diag(a) S dO + k (u . dO);
+            // dS1 = dS + q dO^T;  dk = dS1 u - beta a (S du);
+            // dS' = dS1 - beta k du^T;  da = sum_j dS' S;  dg = da a l';  dS <- Diag(a) dS'
             float udo = 0.f;
 #pragma unroll 4
             for (int s = 0; s < Q; ++s) {
@@ -287,62 +319,29 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
                 udo = fmaf(sm.u[j], sm.dO[j], udo);
             }
             udo = quad_sum(udo);
-            float dk_part;
             {
                 const int i = idx;
-                const float qi = sm.q[i];
-                float sd = 0.f, dsu = 0.f;
+                const float qi = sm.q[i], ai = sm.a[i], bki = bt * sm.k[i];
+                float sd = 0.f, dsu = 0.f, sdu = 0.f, da = 0.f;
 #pragma unroll 4
                 for (int s = 0; s < Q; ++s) {
                     const int j = kParts * s + part;
-                    sd = fmaf(sm.S[i * R + j], sm.dO[j], sd);
-                    const float ds = fmaf(qi, sm.dO[j], sm.dS[i * R + j]);
-                    sm.dS[i * R + j] = ds;
+                    const float sij = sm.S[i * R + j], doj = sm.dO[j], duj = sm.du[j];
+                    sd = fmaf(sij, doj, sd);
+                    const float ds = fmaf(qi, doj, sm.dS[i * R + j]);
                     dsu = fmaf(ds, sm.u[j], dsu);
-                }
-                sd = quad_sum(sd);
-                dk_part = quad_sum(dsu);
-                if (part == 0) IO<T>::st(dq + x + i, fmaf(sm.a[i], sd, sm.k[i] * udo));
-            }
-            __syncthreads();
-            // columns: du = dS^T k;  dv = beta du
-            float dbp = 0.f;
-            {
-                const int j = idx;
-                float d0 = 0.f, d1 = 0.f;
-#pragma unroll 4
-                for (int s = 0; s < Q; s += 2) {
-                    const int i0 = kParts * s + part, i1 = i0 + kParts;
-                    d0 = fmaf(sm.dS[i0 * R + j], sm.k[i0], d0);
-                    d1 = fmaf(sm.dS[i1 * R + j], sm.k[i1], d1);
-                }
-                const float d = quad_sum(d0 + d1);
-                if (part == 0) {
-                    sm.du[j] = d;
-                    IO<T>::st(dv + x + j, bt * d);
-                    dbp = d * sm.w[j];
-                }
-            }
-            __syncthreads();
-            // rows: dk -= beta S' du;  dS' = dS - beta k du^T;  da = sum_j dS' S;
-            // dg = da a l';  dS <- Diag(a) dS'
-            {
-                const int i = idx;
-                const float ai = sm.a[i], bki = bt * sm.k[i];
-                float sdu = 0.f, da = 0.f;
-#pragma unroll 4
-                for (int s = 0; s < Q; ++s) {
-                    const int j = kParts * s + part;
-                    const float sij = sm.S[i * R + j];
-                    sdu = fmaf(sij, sm.du[j], sdu);
-                    const float dsp = fmaf(-bki, sm.du[j], sm.dS[i * R + j]);
+                    sdu = fmaf(sij, duj, sdu);
+                    const float dsp = fmaf(-bki, duj, ds);
                     da = fmaf(dsp, sij, da);
                     sm.dS[i * R + j] = ai * dsp;
                 }
+                sd = quad_sum(sd);
+                dsu = quad_sum(dsu);
                 sdu = quad_sum(sdu);
                 da = quad_sum(da);
                 if (part == 0) {
-                    IO<T>::st(dk + x + i, dk_part - bt * ai * sdu);
+                    IO<T>::st(dq + x + i, fmaf(ai, sd, sm.k[i] * udo));
+                    IO<T>::st(dk + x + i, dsu - bt * ai * sdu);
                     IO<T>::st(dg + x + i, da * ai * sm.lg[i]);
                 }
             }
