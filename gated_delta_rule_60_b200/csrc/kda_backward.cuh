@@ -24,7 +24,9 @@
 // warp and a row pass at most two-way conflicting ones.  A reverse token takes
 // two passes: one over columns, for S'^T k and du, using
 // du = (dS + q dO^T)^T k = dS^T k + dO (q . k) on dS as it enters, and one over
-// rows for everything else.
+// rows for everything else.  A forward token (checkpoint and recompute
+// sweeps) is one pass over columns: the four threads of a column keep their
+// quarter of it in registers between the read and the update.
 #pragma once
 
 #include "kda_common.cuh"
@@ -44,7 +46,7 @@ struct Smem {
     float S[D * kRow];
     float dS[D * kRow];
     static constexpr int kQkParts = D >= 32 ? D / 32 : 1;   // warps holding q and k
-    float q[D], k[D], v[D], a[D], lg[D], dO[D], u[D], w[D], du[D];
+    float q[D], k[D], v[D], a[D], lg[D], dO[D], u[D], du[D];
     float red[threads_of<D>() / 32];
     float qkp[kQkParts];                             // per-warp partial sums of q . k
 };
@@ -194,37 +196,28 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             *reinterpret_cast<float4 *>(sm.S + (e / D) * R + e % D) = pf[u];
         }
     };
-    // column idx of Diag(a) S times k (rows part, part + 4, ...)
-    auto col_ak = [&]() {
-        const int j = idx;
-        float r0 = 0.f, r1 = 0.f;
-#pragma unroll 4
-        for (int s = 0; s < Q; s += 2) {
-            const int i0 = kParts * s + part, i1 = i0 + kParts;
-            r0 = fmaf(sm.a[i0] * sm.S[i0 * R + j], sm.k[i0], r0);
-            r1 = fmaf(sm.a[i1] * sm.S[i1 * R + j], sm.k[i1], r1);
-        }
-        return quad_sum(r0 + r1);
-    };
-    // one forward token on the state in shared memory: w, u, then S <- S_t
+    // one forward token on the state in shared memory, S <- S_t: the four
+    // threads of column j keep their quarter of it in registers, meet in
+    // shuffles for u_j = beta (v_j - ((Diag(a) S)^T k)_j) and update their own
+    // elements, so the token reads and writes S once, with no barrier between
     auto forward_token = [&](float bt) {
         __syncthreads();
-        {
-            const float r = col_ak();
-            if (part == 0) {
-                sm.w[idx] = sm.v[idx] - r;
-                sm.u[idx] = bt * sm.w[idx];
-            }
+        const int j = idx;
+        float col[Q];
+        float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+        for (int s = 0; s < Q; s += 2) {
+            const int i0 = kParts * s + part, i1 = i0 + kParts;
+            col[s] = sm.S[i0 * R + j];
+            col[s + 1] = sm.S[i1 * R + j];
+            r0 = fmaf(sm.a[i0] * col[s], sm.k[i0], r0);
+            r1 = fmaf(sm.a[i1] * col[s + 1], sm.k[i1], r1);
         }
-        __syncthreads();
-        {
-            const int j = idx;
-            const float uj = sm.u[j];
-#pragma unroll 4
-            for (int s = 0; s < Q; ++s) {
-                const int i = kParts * s + part;
-                sm.S[i * R + j] = fmaf(sm.a[i], sm.S[i * R + j], sm.k[i] * uj);
-            }
+        const float uj = bt * (sm.v[j] - quad_sum(r0 + r1));
+#pragma unroll
+        for (int s = 0; s < Q; ++s) {
+            const int i = kParts * s + part;
+            sm.S[i * R + j] = fmaf(sm.a[i], col[s], sm.k[i] * uj);
         }
     };
 

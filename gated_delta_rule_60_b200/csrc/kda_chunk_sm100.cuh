@@ -808,52 +808,35 @@ chunk_fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (tid == 0) KDA_TR(TR_S_BR, c);
                 const int sn = (c + 1) % kSlots;
                 const float4 *g4 = reinterpret_cast<const float4 *>(sm + SM_GAMMA + sn * 512);
-                auto state_quarter = [&](uint32_t (&sv)[32], int qt) {
-                    uint32_t sb[16];
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
-                        const float4 gm = g4[8 * qt + q4];
-                        uint32_t *y = sv + 4 * q4;
-                        const float2 s01 = make_float2(__uint_as_float(y[0]), __uint_as_float(y[1]));
-                        const float2 s23 = make_float2(__uint_as_float(y[2]), __uint_as_float(y[3]));
-                        sb[2 * q4] = pack_bf16(s01.x, s01.y);
-                        sb[2 * q4 + 1] = pack_bf16(s23.x, s23.y);
-                        const float2 g01 = fmul2(make_float2(gm.x, gm.y), s01);
-                        const float2 g23 = fmul2(make_float2(gm.z, gm.w), s23);
-                        y[0] = __float_as_uint(g01.x);
-                        y[1] = __float_as_uint(g01.y);
-                        y[2] = __float_as_uint(g23.x);
-                        y[3] = __float_as_uint(g23.y);
-                    }
-                    tmem_st16(tm + la + COL_S16 + 16 * qt, sb);
-                    tmem_st16(tm + la + COL_S + 32 * qt, *reinterpret_cast<uint32_t(*)[16]>(sv));
-                    tmem_st16(tm + la + COL_S + 32 * qt + 16, *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
-                };
-                if (has_next && ready) {
-                    // double-buffered: quarter qt + 1 loads while quarter qt is
-                    // scaled and converted; O is read last
-                    uint32_t sa[32], sb2[32];
-                    tmem_ld32(tm + la + COL_S, sa);
-                    tmem_wait_ld();
-                    tmem_ld32(tm + la + COL_S + 32, sb2);
-                    state_quarter(sa, 0);
-                    tmem_wait_ld();
-                    tmem_ld32(tm + la + COL_S + 64, sa);
-                    state_quarter(sb2, 1);
-                    tmem_wait_ld();
-                    tmem_ld32(tm + la + COL_S + 96, sb2);
-                    state_quarter(sa, 2);
-                    tmem_wait_ld();
-                    tmem_ld32(tm + la + COL_O, ov);
-                    state_quarter(sb2, 3);
-                } else {
-                    // the last step: O and the final state
-                    tmem_ld32(tm + la + COL_O, ov);
+                tmem_ld32(tm + la + COL_O, ov);      // waited for with the first quarter
 #pragma unroll 1
-                    for (int qt = 0; qt < 4 && ready && ch.hT; ++qt) {
-                        uint32_t sv[32];
-                        tmem_ld32(tm + la + COL_S + 32 * qt, sv);
-                        tmem_wait_ld();
+                for (int qt = 0; qt < 4 && ready; ++qt) {       // 32 key channels at a time
+                    uint32_t sv[32];
+                    tmem_ld32(tm + la + COL_S + 32 * qt, sv);
+                    tmem_wait_ld();
+                    if (tid == 0 && qt == 0) KDA_TR(TR_S_LD, c);
+                    if (has_next) {
+                        uint32_t sb[16];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 gm = g4[8 * qt + q4];
+                            uint32_t *y = sv + 4 * q4;
+                            const float2 s01 = make_float2(__uint_as_float(y[0]), __uint_as_float(y[1]));
+                            const float2 s23 = make_float2(__uint_as_float(y[2]), __uint_as_float(y[3]));
+                            sb[2 * q4] = pack_bf16(s01.x, s01.y);
+                            sb[2 * q4 + 1] = pack_bf16(s23.x, s23.y);
+                            const float2 g01 = fmul2(make_float2(gm.x, gm.y), s01);
+                            const float2 g23 = fmul2(make_float2(gm.z, gm.w), s23);
+                            y[0] = __float_as_uint(g01.x);
+                            y[1] = __float_as_uint(g01.y);
+                            y[2] = __float_as_uint(g23.x);
+                            y[3] = __float_as_uint(g23.y);
+                        }
+                        tmem_st16(tm + la + COL_S16 + 16 * qt, sb);
+                        tmem_st16(tm + la + COL_S + 32 * qt, *reinterpret_cast<uint32_t(*)[16]>(sv));
+                        tmem_st16(tm + la + COL_S + 32 * qt + 16, *reinterpret_cast<uint32_t(*)[16]>(sv + 16));
+                        if (tid == 0) KDA_TR(qt == 1 ? TR_S_H0 : TR_S_H1, c);
+                    } else if (ch.hT) {
                         OutRegs srr;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) srr.v[i] = sv[i];
