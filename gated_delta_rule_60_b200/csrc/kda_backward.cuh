@@ -21,7 +21,10 @@
 // of the current pass, each a quarter of it (every fourth element), and meet
 // in two shuffles; the CTA has 4 d threads.  State rows are padded to d + 8
 // floats in shared memory, so that a column pass reads 32 distinct banks per
-// warp and a row pass at most two-way conflicting ones.  A reverse token takes
+// warp; in a row pass, rows 4-7 of a warp's eight walk their columns in a
+// permuted order, which makes it conflict-free too.  Shared memory is the
+// limit of this kernel: every warp-wide access costs a wavefront, even a
+// broadcast of a few vector elements, so vectors read together are packed.  A reverse token takes
 // two passes: one over columns, for S'^T k and du, using
 // du = (dS + q dO^T)^T k = dS^T k + dO (q . k) on dS as it enters, and one over
 // rows for everything else.  A forward token (checkpoint and recompute
@@ -46,7 +49,12 @@ struct Smem {
     float S[D * kRow];
     float dS[D * kRow];
     static constexpr int kQkParts = D >= 32 ? D / 32 : 1;   // warps holding q and k
-    float q[D], k[D], v[D], a[D], lg[D], dO[D], u[D], du[D];
+    // vectors read together are packed, one shared-memory access each:
+    // ak[i] = (a_i, k_i) in the column passes, vec[j] = (dO_j, du_j, u_j, -)
+    // in the row pass
+    float4 vec[D];
+    float2 ak[D];
+    float q[D], v[D], lg[D];
     float red[threads_of<D>() / 32];
     float qkp[kQkParts];                             // per-warp partial sums of q . k
 };
@@ -175,11 +183,10 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         if (tid < D) {
             const float s = sigmoid_acc(r.g);
             sm.q[tid] = r.q;
-            sm.k[tid] = r.k;
             sm.v[tid] = r.v;
-            sm.a[tid] = expf(-5.f * s);
+            sm.ak[tid] = make_float2(expf(-5.f * s), r.k);
             sm.lg[tid] = -5.f * s * (1.f - s);
-            sm.dO[tid] = r.dO;
+            sm.vec[tid].x = r.dO;
         }
     };
     // one token state (D x D fp32) through registers, 16 bytes per access
@@ -210,14 +217,16 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             const int i0 = kParts * s + part, i1 = i0 + kParts;
             col[s] = sm.S[i0 * R + j];
             col[s + 1] = sm.S[i1 * R + j];
-            r0 = fmaf(sm.a[i0] * col[s], sm.k[i0], r0);
-            r1 = fmaf(sm.a[i1] * col[s + 1], sm.k[i1], r1);
+            const float2 ak0 = sm.ak[i0], ak1 = sm.ak[i1];
+            r0 = fmaf(ak0.x * col[s], ak0.y, r0);
+            r1 = fmaf(ak1.x * col[s + 1], ak1.y, r1);
         }
         const float uj = bt * (sm.v[j] - quad_sum(r0 + r1));
 #pragma unroll
         for (int s = 0; s < Q; ++s) {
             const int i = kParts * s + part;
-            sm.S[i * R + j] = fmaf(sm.a[i], col[s], sm.k[i] * uj);
+            const float2 ak = sm.ak[i];
+            sm.S[i * R + j] = fmaf(ak.x, col[s], ak.y * uj);
         }
     };
 
@@ -283,20 +292,20 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
 #pragma unroll 4
                 for (int s = 0; s < Q; s += 2) {
                     const int i0 = kParts * s + part, i1 = i0 + kParts;
-                    const float k0 = sm.k[i0], k1 = sm.k[i1];
-                    r0 = fmaf(sm.a[i0] * sm.S[i0 * R + j], k0, r0);
-                    r1 = fmaf(sm.a[i1] * sm.S[i1 * R + j], k1, r1);
-                    d0 = fmaf(sm.dS[i0 * R + j], k0, d0);
-                    d1 = fmaf(sm.dS[i1 * R + j], k1, d1);
+                    const float2 ak0 = sm.ak[i0], ak1 = sm.ak[i1];
+                    r0 = fmaf(ak0.x * sm.S[i0 * R + j], ak0.y, r0);
+                    r1 = fmaf(ak1.x * sm.S[i1 * R + j], ak1.y, r1);
+                    d0 = fmaf(sm.dS[i0 * R + j], ak0.y, d0);
+                    d1 = fmaf(sm.dS[i1 * R + j], ak1.y, d1);
                 }
                 const float r = quad_sum(r0 + r1), dsk = quad_sum(d0 + d1);
                 if (part == 0) {
                     float qk = 0.f;
 #pragma unroll
                     for (int p = 0; p < Smem<D>::kQkParts; ++p) qk += sm.qkp[p];
-                    const float wj = sm.v[j] - r, du = fmaf(sm.dO[j], qk, dsk);
-                    sm.u[j] = bt * wj;
-                    sm.du[j] = du;
+                    const float wj = sm.v[j] - r, du = fmaf(sm.vec[j].x, qk, dsk);
+                    sm.vec[j].y = du;
+                    sm.vec[j].z = bt * wj;
                     IO<T>::st(dv + x + j, bt * du);
                     dbp = du * wj;
                 }
@@ -305,26 +314,25 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
             // rows, one pass: dq = S_t dO = Diag(a) S dO + k (u . dO);
             // dS1 = dS + q dO^T;  dk = dS1 u - beta a (S du);
             // dS' = dS1 - beta k du^T;  da = sum_j dS' S;  dg = da a l';  dS <- Diag(a) dS'
-            float udo = 0.f;
-#pragma unroll 4
-            for (int s = 0; s < Q; ++s) {
-                const int j = kParts * s + part;
-                udo = fmaf(sm.u[j], sm.dO[j], udo);
-            }
-            udo = quad_sum(udo);
             {
-                const int i = idx;
-                const float qi = sm.q[i], ai = sm.a[i], bki = bt * sm.k[i];
-                float sd = 0.f, dsu = 0.f, sdu = 0.f, da = 0.f;
+                // rows 4-7 of each group of eight (one warp) walk their columns
+                // in the order s ^ 1, so that a warp's 32 lanes hit 32 banks
+                const int i = idx, flip = (idx >> 2) & 1;
+                const float qi = sm.q[i];
+                const float2 aki = sm.ak[i];
+                const float ai = aki.x, bki = bt * aki.y;
+                float sd = 0.f, dsu = 0.f, sdu = 0.f, da = 0.f, udo = 0.f;
 #pragma unroll 4
                 for (int s = 0; s < Q; ++s) {
-                    const int j = kParts * s + part;
-                    const float sij = sm.S[i * R + j], doj = sm.dO[j], duj = sm.du[j];
-                    sd = fmaf(sij, doj, sd);
-                    const float ds = fmaf(qi, doj, sm.dS[i * R + j]);
-                    dsu = fmaf(ds, sm.u[j], dsu);
-                    sdu = fmaf(sij, duj, sdu);
-                    const float dsp = fmaf(-bki, duj, ds);
+                    const int j = kParts * (s ^ flip) + part;
+                    const float4 vj = sm.vec[j];             // dO_j, du_j, u_j
+                    const float sij = sm.S[i * R + j];
+                    udo = fmaf(vj.z, vj.x, udo);
+                    sd = fmaf(sij, vj.x, sd);
+                    const float ds = fmaf(qi, vj.x, sm.dS[i * R + j]);
+                    dsu = fmaf(ds, vj.z, dsu);
+                    sdu = fmaf(sij, vj.y, sdu);
+                    const float dsp = fmaf(-bki, vj.y, ds);
                     da = fmaf(dsp, sij, da);
                     sm.dS[i * R + j] = ai * dsp;
                 }
@@ -332,8 +340,9 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
                 dsu = quad_sum(dsu);
                 sdu = quad_sum(sdu);
                 da = quad_sum(da);
+                udo = quad_sum(udo);
                 if (part == 0) {
-                    IO<T>::st(dq + x + i, fmaf(ai, sd, sm.k[i] * udo));
+                    IO<T>::st(dq + x + i, fmaf(ai, sd, aki.y * udo));
                     IO<T>::st(dk + x + i, dsu - bt * ai * sdu);
                     IO<T>::st(dg + x + i, da * ai * sm.lg[i]);
                 }
