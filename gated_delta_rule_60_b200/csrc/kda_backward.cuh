@@ -211,22 +211,23 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         __syncthreads();
         const int j = idx;
         float col[Q];
+        float2 akr[Q];
         float r0 = 0.f, r1 = 0.f;
 #pragma unroll
         for (int s = 0; s < Q; s += 2) {
             const int i0 = kParts * s + part, i1 = i0 + kParts;
             col[s] = sm.S[i0 * R + j];
             col[s + 1] = sm.S[i1 * R + j];
-            const float2 ak0 = sm.ak[i0], ak1 = sm.ak[i1];
-            r0 = fmaf(ak0.x * col[s], ak0.y, r0);
-            r1 = fmaf(ak1.x * col[s + 1], ak1.y, r1);
+            akr[s] = sm.ak[i0];
+            akr[s + 1] = sm.ak[i1];
+            r0 = fmaf(akr[s].x * col[s], akr[s].y, r0);
+            r1 = fmaf(akr[s + 1].x * col[s + 1], akr[s + 1].y, r1);
         }
         const float uj = bt * (sm.v[j] - quad_sum(r0 + r1));
 #pragma unroll
         for (int s = 0; s < Q; ++s) {
             const int i = kParts * s + part;
-            const float2 ak = sm.ak[i];
-            sm.S[i * R + j] = fmaf(ak.x, col[s], ak.y * uj);
+            sm.S[i * R + j] = fmaf(akr[s].x, col[s], akr[s].y * uj);
         }
     };
 
