@@ -24,12 +24,12 @@
 // warp; in a row pass, rows 4-7 of a warp's eight walk their columns in a
 // permuted order, which makes it conflict-free too.  Shared memory is the
 // limit of this kernel: every warp-wide access costs a wavefront, even a
-// broadcast of a few vector elements, so vectors read together are packed.  A reverse token takes
-// two passes: one over columns, for S'^T k and du, using
-// du = (dS + q dO^T)^T k = dS^T k + dO (q . k) on dS as it enters, and one over
-// rows for everything else.  A forward token (checkpoint and recompute
-// sweeps) is one pass over columns: the four threads of a column keep their
-// quarter of it in registers between the read and the update.
+// broadcast of a few vector elements, so vectors read together are packed.
+// A reverse token takes two passes: one over columns, for S'^T k and du,
+// using du = (dS + q dO^T)^T k = dS^T k + dO (q . k) on dS as it enters, and
+// one over rows for everything else.  A forward token (checkpoint and
+// recompute sweeps) is one pass over columns: the four threads of a column
+// keep their quarter of it in registers between the read and the update.
 #pragma once
 
 #include "kda_common.cuh"
@@ -68,7 +68,8 @@ __device__ __forceinline__ float quad_sum(float x) {
 
 // Copies between a padded shared-memory matrix and a dense D x D global
 // array, 16 bytes per access, up to eight global loads in flight per thread
-// (the reverse sweep moves one 64 KB state per token).
+// (h0, dhT, the checkpoints and the recomputed token states; the reverse
+// pass fetches its token states one token ahead instead).
 template <int D>
 __device__ __forceinline__ void mat_from_global(float *sdst, const float *__restrict__ src, int tid) {
     constexpr int R = Smem<D>::kRow, N4 = D * D / 4, NT = threads_of<D>(), B = 8;
