@@ -59,6 +59,30 @@ def test_workspace_size_is_host_only(lib):
     assert ws >= 0
 
 
+def _segment_workspace(G, seg0, T, H):
+    # G start states, G transfer matrices and G end states of 128 x 128 fp32
+    # per head, plus one bf16 row of M^T q per token and head after segment 0
+    return 3 * G * H * 128 * 128 * 4 + (T - seg0) * H * 128 * 2
+
+
+def test_segment_plans_of_the_long_context_workloads(lib):
+    """The segment plans the long-sequence path picks on a 148-SM B200, read
+    back through the workspace they need: at 2^20 tokens, 16 heads five equal
+    segments of 209,728 tokens (the last one 209,664; 144 CTAs in the local
+    pass, one wave); at 8 heads eighteen segments of 55,200 tokens with
+    segment 0 twice as long.  Below 8,192 tokens, with several sequences,
+    and when the heads alone fill the SMs there is no split."""
+    ws = lambda N, T, H: lib.kda_chunk_fwd_workspace_size(N, T, H, 128, 128, 0)
+    T = 1 << 20
+    assert ws(1, T, 16) == _segment_workspace(5, 209728, T, 16)
+    assert 4 * 209728 + 209664 == T
+    assert ws(1, T, 8) == _segment_workspace(18, 2 * 55200, T, 8)
+    assert 2 * 55200 + 16 * 55200 + 54976 == T
+    assert ws(1, 8191, 2) == 0
+    assert ws(2, 1 << 15, 2) == 0
+    assert ws(1, T, 96) == 0 and ws(1, T, 148) == 0
+
+
 def _call_fwd(lib, **over):
     args = dict(q=16, k=16, v=16, g=16, beta=16, h0=None, cu=None, N=1, T=32,
                 H=2, dk=16, dv=16, dt=1, o=16, hT=None, ws=None, wsb=0,
