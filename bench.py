@@ -288,6 +288,14 @@ def run_gpu(args):
             print(json.dumps({"only": "decode", "decode": decode}))
         return 0
 
+    if args.only == "backward":
+        stream = torch.cuda.Stream(device=dev)
+        torch.cuda.synchronize()
+        backward = _measure_backward(dev, stream, args, world, binding, inputs)
+        if rank == 0:
+            print(json.dumps({"only": "backward", "backward": backward}))
+        return 0
+
     # ---------------- prefill workload ----------------
     w = workloads.K3_PREFILL
     inp = w.make()
@@ -632,8 +640,9 @@ def main():
                     help="skip the decode measurement")
     ap.add_argument("--skip-workloads", action="store_true",
                     help="skip the varlen and long-context prefill measurements")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
-                    help="run one part only (for profiling): the K3 prefill or the decode")
+    ap.add_argument("--only", choices=["prefill", "decode", "backward"], default=None,
+                    help="run one part only (for profiling): the K3 prefill, the decode "
+                         "or the backward")
     ap.add_argument("--record-traffic", metavar="NCU_CSV", default=None,
                     help="write the prefill DRAM traffic record from an ncu --csv log of "
                          "dram__bytes_read.sum and dram__bytes_write.sum (no GPU needed)")
