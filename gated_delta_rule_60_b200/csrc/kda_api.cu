@@ -155,7 +155,7 @@ kda_status dispatch_decode(int d, const void *q, const void *k, const void *v,
 
 extern "C" {
 
-int32_t kda_version(void) { return 10000; }
+int32_t kda_version(void) { return 10100; }
 
 const char *kda_status_string(kda_status s) {
     switch (s) {
