@@ -379,6 +379,8 @@ def run_gpu(args):
             torch.cuda.empty_cache()
         extra["backward_2k"] = _measure_backward(dev, stream, args, world, binding, inputs)
         torch.cuda.empty_cache()
+        extra.update(_measure_layer_rows(dev, stream, world, hbm_peak, kern_ms, binding,
+                                         inputs))
     decode = None
     if not args.skip_decode:
         decode = _measure_decode(dev, stream, args, world, hbm_peak, binding, inputs, workloads)
@@ -463,6 +465,106 @@ def _measure_backward(dev, stream, args, world, binding, inputs):
     return {"tokens": T, "heads": H, "sequences": 1, "ms": ms,
             "Mtok_s": world * T / (ms * 1e-3) / 1e6, "fp32_tflops": tflops,
             "frac_of_fp32_peak": tflops / FP32_PEAK_TFLOPS, "launches_per_step": 1}
+
+
+# algorithmic bytes per (token, head) of the prologue at d = 128: xq, xk, xv
+# and beta_raw read, q, k, v and beta written, bf16
+PROLOGUE_BYTES_PER_TOKEN_HEAD = 2 * 3 * 128 * 2 + 2 * 2     # 1540
+# the gated prefill reads z as well
+GATED_BYTES_PER_TOKEN_HEAD = BYTES_PER_TOKEN_HEAD + 128 * 2  # 1538
+
+
+def _events_ms(stream, fn, warmup, steps):
+    """Mean device time of fn() over `steps` launches on `stream` (CUDA
+    events), after `warmup` untimed launches."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            fn()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _prologue_local(dev, stream, binding, inputs):
+    T, H, d = 8192, 96, 128
+    li = inputs.make_layer([T], H, d, torch.bfloat16, seed=1011, device=dev)
+    torch.cuda.synchronize()
+    ms = _events_ms(stream, lambda: binding.kda_prologue(
+        li.xq, li.xk, li.xv, li.wq, li.wk, li.wv, li.beta_raw, li.cu_seqlens,
+        stream=stream), 3, 10)
+    alg = T * H * PROLOGUE_BYTES_PER_TOKEN_HEAD + 3 * H * d * 4 * 4
+    return ms, alg, T, H
+
+
+def _gated_local(dev, stream, binding, inputs):
+    T, H, d = 8192, 96, 128
+    pre = inputs.make_prefill([T], H, d, d, torch.bfloat16, 1012, device=dev)
+    gen = torch.Generator(device=dev).manual_seed(6)
+    z = torch.randn(T, H, d, generator=gen, device=dev).to(torch.bfloat16)
+    o = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+    hT = torch.empty(1, H, d, d, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    ms = _events_ms(stream, lambda: binding.kda_chunk_fwd_gated(
+        pre.q, pre.k, pre.v, pre.g, pre.beta, z, None, pre.cu_seqlens, o=o, hT=hT,
+        stream=stream), 3, 10)
+    alg = T * H * GATED_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    return ms, alg, T, H
+
+
+def _softplus_local(dev, stream, binding, inputs):
+    T, H, d = 2048, 96, 128
+    pre = inputs.make_prefill([T], H, d, d, torch.bfloat16, 1013, 0.02, device=dev)
+    o = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+    hT = torch.empty(1, H, d, d, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    ms = _events_ms(stream, lambda: binding.kda_chunk_fwd_softplus(
+        pre.q, pre.k, pre.v, pre.g, pre.beta, pre.h0, pre.cu_seqlens, o=o, hT=hT,
+        stream=stream), 1, 3)
+    alg = T * H * BYTES_PER_TOKEN_HEAD + 2 * H * STATE_BYTES
+    return ms, alg, T, H
+
+
+def _measure_layer_rows(dev, stream, world, hbm_peak, plain_ms, binding, inputs):
+    """The rows around the operator, each in one launch per step:
+    - prologue_k3: kda_prologue on the K3 shape (96 heads x 8,192 tokens,
+      d = 128, bf16), a memory-bound pass;
+    - gated_k3: kda_chunk_fwd_gated on the K3 shape (the output gate fused
+      into the tensor-core prefill), with its cost over the plain launch;
+    - softplus_2k: kda_chunk_fwd_softplus on 96 heads x 2,048 tokens (the
+      unbounded gate on the fp32 CUDA-core kernel, a correctness path).
+    Each rank measures on its own; a failure is reported in the row instead
+    of ending the run, and every rank takes the same collective steps."""
+    rows = {}
+    for name, fn in (("prologue_k3", _prologue_local), ("gated_k3", _gated_local),
+                     ("softplus_2k", _softplus_local)):
+        _barrier(world)
+        err = None
+        try:
+            ms, alg, T, H = fn(dev, stream, binding, inputs)
+            st = binding.kda_stream_status(stream)
+            if st != binding.KDA_OK:
+                err = "kernel status: " + binding.kda_status_string(st)
+        except Exception as e:                      # reported in the JSON line
+            err = "%s: %s" % (type(e).__name__, e)
+        ms = _max_over_ranks(float("inf") if err else ms, world)
+        if err or ms == float("inf"):
+            rows[name] = {"error": err or "failed on another rank"}
+        else:
+            gbs = alg / (ms * 1e-3) / 1e9
+            rows[name] = {"tokens": T, "heads": H, "ms": ms,
+                          "Mtok_s": world * T / (ms * 1e-3) / 1e6, "hbm_gbs": gbs,
+                          "frac_of_peak": gbs / hbm_peak,
+                          "algorithmic_bytes_per_launch": alg, "launches_per_step": 1}
+        torch.cuda.empty_cache()
+    if "ms" in rows.get("gated_k3", {}):
+        rows["gated_k3"]["cost_over_plain"] = rows["gated_k3"]["ms"] / plain_ms - 1.0
+    return rows
 
 
 def _measure_e2e(inp, dev, cu, o, hT, ws, stream, args, world, T, H, d, binding):

@@ -131,3 +131,106 @@ def test_traffic_record_round_trip(tmp_path, monkeypatch):
     assert bench._measured_traffic() == pytest.approx(809.6e6 + 186.4e6)
     monkeypatch.setattr(bench, "_prefill_source_hash", lambda: "0" * 16)
     assert bench._measured_traffic() is None
+
+
+def test_layer_rows_report_and_isolate_failures(monkeypatch):
+    """The bench's rows for the prologue, the gated prefill and the softplus
+    variant: a measured row carries its time, throughput and roofline
+    fraction; a row whose call raises, or whose kernel reports a bad status,
+    carries the error instead, and the others are still measured."""
+    import bench
+
+    class FakeBinding:
+        KDA_OK = 0
+        status = [0, 5]          # OK after the prologue, a timeout after the gated call
+
+        def kda_stream_status(self, stream=None):
+            return self.status.pop(0)
+
+        def kda_status_string(self, st):
+            return "a kernel's bounded wait ran out"
+
+    def prologue(dev, stream, binding, inputs):
+        return 0.25, 1_000_000_000, 8192, 96
+
+    def gated(dev, stream, binding, inputs):
+        return 0.8, 1_200_000_000, 8192, 96
+
+    def softplus(dev, stream, binding, inputs):
+        raise RuntimeError("no such kernel")
+
+    monkeypatch.setattr(bench, "_prologue_local", prologue)
+    monkeypatch.setattr(bench, "_gated_local", gated)
+    monkeypatch.setattr(bench, "_softplus_local", softplus)
+    rows = bench._measure_layer_rows("cpu", None, 1, 8000.0, 0.7, FakeBinding(), None)
+    p = rows["prologue_k3"]
+    assert p["ms"] == 0.25 and p["hbm_gbs"] == pytest.approx(4000.0)
+    assert p["frac_of_peak"] == pytest.approx(0.5)
+    assert p["Mtok_s"] == pytest.approx(8192 / 0.25e-3 / 1e6)
+    assert rows["gated_k3"] == {"error": "kernel status: a kernel's bounded wait ran out"}
+    assert rows["softplus_2k"]["error"].startswith("RuntimeError: no such kernel")
+
+
+def test_gated_row_reports_its_cost_over_the_plain_launch(monkeypatch):
+    import bench
+
+    class FakeBinding:
+        KDA_OK = 0
+
+        def kda_stream_status(self, stream=None):
+            return 0
+
+    for name in ("_prologue_local", "_gated_local", "_softplus_local"):
+        monkeypatch.setattr(bench, name, lambda *a: (0.77, 10**9, 8192, 96))
+    rows = bench._measure_layer_rows("cpu", None, 1, 8000.0, 0.7, FakeBinding(), None)
+    assert rows["gated_k3"]["cost_over_plain"] == pytest.approx(0.1)
+    assert "cost_over_plain" not in rows["prologue_k3"]
+    json.dumps(rows)
+
+
+class _OkBinding:
+    KDA_OK = 0
+
+    def kda_stream_status(self, stream=None):
+        return 0
+
+
+def _layer_rank_main(rank, world, port, out_dir):
+    """One rank of the layer-row measurement: rank 0's gated call fails, every
+    other call succeeds with a rank-dependent time."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        def ok(*a):
+            return 0.5 + rank, 10**9, 8192, 96
+
+        def gated(*a):
+            if rank == 0:
+                raise RuntimeError("launch failed")
+            return ok()
+
+        bench._prologue_local, bench._gated_local, bench._softplus_local = ok, gated, ok
+        rows = bench._measure_layer_rows("cpu", None, world, 8000.0, 0.7, _OkBinding(), None)
+        with open(os.path.join(out_dir, "layer%d.json" % rank), "w") as f:
+            json.dump(rows, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_layer_rows_world2_gloo_one_rank_fails(tmp_path):
+    """Every rank takes the same collective steps: a call that fails on one
+    rank ends as an error row on all ranks (no rank waits for good), and the
+    rows that succeed everywhere report the slowest rank's time."""
+    world = 2
+    mp.start_processes(_layer_rank_main, args=(world, _free_port(), str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    for r in range(world):
+        with open(tmp_path / ("layer%d.json" % r)) as f:
+            rows = json.load(f)
+        assert rows["prologue_k3"]["ms"] == 1.5 and rows["softplus_2k"]["ms"] == 1.5
+        assert "error" in rows["gated_k3"]
+    with open(tmp_path / "layer1.json") as f:
+        assert json.load(f)["gated_k3"] == {"error": "failed on another rank"}
