@@ -467,13 +467,6 @@ def _measure_backward(dev, stream, args, world, binding, inputs):
             "frac_of_fp32_peak": tflops / FP32_PEAK_TFLOPS, "launches_per_step": 1}
 
 
-# algorithmic bytes per (token, head) of the prologue at d = 128: xq, xk, xv
-# and beta_raw read, q, k, v and beta written, bf16
-PROLOGUE_BYTES_PER_TOKEN_HEAD = 2 * 3 * 128 * 2 + 2 * 2     # 1540
-# the gated prefill reads z as well
-GATED_BYTES_PER_TOKEN_HEAD = BYTES_PER_TOKEN_HEAD + 128 * 2  # 1538
-
-
 def _events_ms(stream, fn, warmup, steps):
     """Mean device time of fn() over `steps` launches on `stream` (CUDA
     events), after `warmup` untimed launches."""
@@ -491,19 +484,26 @@ def _events_ms(stream, fn, warmup, steps):
     return e0.elapsed_time(e1) / steps
 
 
+# (tokens, heads, head size) of the rows around the operator
+LAYER_ROW_SHAPES = {"prologue_k3": (8192, 96, 128), "gated_k3": (8192, 96, 128),
+                    "softplus_2k": (2048, 96, 128)}
+
+
 def _prologue_local(dev, stream, binding, inputs):
-    T, H, d = 8192, 96, 128
+    T, H, d = LAYER_ROW_SHAPES["prologue_k3"]
     li = inputs.make_layer([T], H, d, torch.bfloat16, seed=1011, device=dev)
     torch.cuda.synchronize()
     ms = _events_ms(stream, lambda: binding.kda_prologue(
         li.xq, li.xk, li.xv, li.wq, li.wk, li.wv, li.beta_raw, li.cu_seqlens,
         stream=stream), 3, 10)
-    alg = T * H * PROLOGUE_BYTES_PER_TOKEN_HEAD + 3 * H * d * 4 * 4
+    # xq, xk, xv, beta_raw read and q, k, v, beta written (bf16; 1,540 B per
+    # (token, head) at d = 128), plus the fp32 taps
+    alg = T * H * (2 * 3 * d * 2 + 2 * 2) + 3 * H * d * 4 * 4
     return ms, alg, T, H
 
 
 def _gated_local(dev, stream, binding, inputs):
-    T, H, d = 8192, 96, 128
+    T, H, d = LAYER_ROW_SHAPES["gated_k3"]
     pre = inputs.make_prefill([T], H, d, d, torch.bfloat16, 1012, device=dev)
     gen = torch.Generator(device=dev).manual_seed(6)
     z = torch.randn(T, H, d, generator=gen, device=dev).to(torch.bfloat16)
@@ -513,12 +513,13 @@ def _gated_local(dev, stream, binding, inputs):
     ms = _events_ms(stream, lambda: binding.kda_chunk_fwd_gated(
         pre.q, pre.k, pre.v, pre.g, pre.beta, z, None, pre.cu_seqlens, o=o, hT=hT,
         stream=stream), 3, 10)
-    alg = T * H * GATED_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    # the prefill's bytes plus z (1,538 B per (token, head) at d = 128) and hT
+    alg = T * H * ((5 * d + d) * 2 + 2) + H * d * d * 4
     return ms, alg, T, H
 
 
 def _softplus_local(dev, stream, binding, inputs):
-    T, H, d = 2048, 96, 128
+    T, H, d = LAYER_ROW_SHAPES["softplus_2k"]
     pre = inputs.make_prefill([T], H, d, d, torch.bfloat16, 1013, 0.02, device=dev)
     o = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
     hT = torch.empty(1, H, d, d, dtype=torch.float32, device=dev)
@@ -526,7 +527,8 @@ def _softplus_local(dev, stream, binding, inputs):
     ms = _events_ms(stream, lambda: binding.kda_chunk_fwd_softplus(
         pre.q, pre.k, pre.v, pre.g, pre.beta, pre.h0, pre.cu_seqlens, o=o, hT=hT,
         stream=stream), 1, 3)
-    alg = T * H * BYTES_PER_TOKEN_HEAD + 2 * H * STATE_BYTES
+    # the prefill's bytes (1,282 B per (token, head) at d = 128), h0 and hT
+    alg = T * H * ((4 * d + d) * 2 + 2) + 2 * H * d * d * 4
     return ms, alg, T, H
 
 

@@ -234,3 +234,47 @@ def test_layer_rows_world2_gloo_one_rank_fails(tmp_path):
         assert "error" in rows["gated_k3"]
     with open(tmp_path / "layer1.json") as f:
         assert json.load(f)["gated_k3"] == {"error": "failed on another rank"}
+
+
+def test_layer_row_calls_bind_to_the_binding(monkeypatch):
+    """The three row measurements call the real binding's functions with
+    arguments that bind to their signatures, tensors of the shapes the
+    binding checks, and the keyword stream: checked on small shapes on the
+    CPU with a stand-in that records each call instead of launching."""
+    import inspect
+    import bench
+    from gated_delta_rule_60_b200 import binding as real, inputs
+
+    calls = []
+
+    class Recorder:
+        KDA_OK = 0
+
+        def __getattr__(self, name):
+            fn = getattr(real, name)
+
+            def record(*a, **kw):
+                bound = inspect.signature(fn).bind(*a, **kw)
+                calls.append((name, bound.arguments))
+            return record
+
+    monkeypatch.setattr(bench, "LAYER_ROW_SHAPES", {"prologue_k3": (40, 3, 16),
+                                                    "gated_k3": (40, 3, 16),
+                                                    "softplus_2k": (24, 2, 32)})
+    monkeypatch.setattr(bench, "_events_ms", lambda stream, fn, w, s: (fn(), 1.0)[1])
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    stream = object()
+    for fn in (bench._prologue_local, bench._gated_local, bench._softplus_local):
+        fn("cpu", stream, Recorder(), inputs)
+    names = [c[0] for c in calls]
+    assert names == ["kda_prologue", "kda_chunk_fwd_gated", "kda_chunk_fwd_softplus"]
+    pro, gated, soft = (c[1] for c in calls)
+    assert pro["xq"].shape == (40, 3, 16) and pro["wq"].shape == (3, 16, 4)
+    assert pro["beta_raw"].shape == (40, 3) and pro["cu_seqlens"].tolist() == [0, 40]
+    assert gated["z"].shape == gated["v"].shape == gated["o"].shape == (40, 3, 16)
+    assert gated["hT"].shape == (1, 3, 16, 16) and gated["h0"] is None
+    assert soft["h0"].shape == soft["hT"].shape == (1, 2, 32, 32)
+    for args in (pro, gated, soft):
+        assert args["stream"] is stream
+        assert all(t.dtype in (torch.bfloat16, torch.float32, torch.int32)
+                   for t in args.values() if isinstance(t, torch.Tensor))
