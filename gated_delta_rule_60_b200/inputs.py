@@ -2,8 +2,11 @@
 
 This module draws random numbers and nothing else: it holds none of the
 operator's arithmetic, so the tests, the benchmark and the fp64 oracle can all
-take their inputs from it.  Everything is drawn on the CPU with a seeded
-``torch.Generator`` and returned as CPU tensors.
+take their inputs from it.  By default everything is drawn on the CPU with a
+seeded ``torch.Generator`` and returned as CPU tensors; with ``device`` set,
+make_prefill, make_decode_step and make_layer draw with that device's
+generator instead (same distributions, a different random stream) and return
+tensors there.
 
 Distributions (the workloads of the KDA operator description):
   q, k ~ N(0, 1), then L2-normalised per (token, head) over the key channels;
