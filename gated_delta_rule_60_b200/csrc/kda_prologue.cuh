@@ -144,10 +144,11 @@ prologue_kernel(const T *__restrict__ xq, const T *__restrict__ xk, const T *__r
         n = seq_of(cu, N, T_tot, t0);
         s_begin = seq_start(cu, N, T_tot, n);
         s_end = seq_start(cu, N, T_tot, n + 1);
+        // (tp >= 0 as well: a malformed cu_seqlens may give a negative start)
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
             const int64_t tp = t0 - 1 - i;
-            if (tp >= s_begin) Vec8<T>::ld(x + (size_t)tp * row + col, hist[i]);
+            if (tp >= s_begin && tp >= 0) Vec8<T>::ld(x + (size_t)tp * row + col, hist[i]);
         }
     }
 
