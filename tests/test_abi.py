@@ -241,3 +241,33 @@ def test_backward_workspace_and_arguments(lib):
         [P(256)] * 5 + [None]
     assert lib.kda_chunk_bwd(*args, None, 0, None) == binding.KDA_ERR_WORKSPACE
     assert lib.kda_chunk_bwd(*args, P(512), 16, None) == binding.KDA_ERR_WORKSPACE
+
+
+def test_softplus_entry_points_checked_on_the_host(lib):
+    """The unbounded-gate prefill and decode refuse unsupported head sizes and
+    dtypes, bad counts, and NULL or misaligned pointers before any launch
+    (the pointers below are never dereferenced)."""
+    P = ctypes.c_void_p
+    INV, UNS, OK = binding.KDA_ERR_INVALID_ARGUMENT, binding.KDA_ERR_UNSUPPORTED, binding.KDA_OK
+
+    def fwd(N=1, T=64, H=2, d=128, dt=binding.KDA_BF16, q=256, cu=None, o=256):
+        p = lambda x: None if x is None else P(x)
+        return lib.kda_chunk_fwd_softplus(p(q), P(256), P(256), P(256), P(256), None, p(cu),
+                                          N, T, H, d, d, dt, p(o), None, None)
+
+    assert fwd(d=48) == UNS and fwd(dt=7) == UNS
+    assert fwd(H=0) == INV and fwd(N=-1) == INV and fwd(T=-1) == INV
+    assert fwd(N=0, T=64) == INV and fwd(N=0, T=0) == OK
+    assert fwd(N=3, T=64) == INV                  # equal lengths need T % N == 0
+    assert fwd(q=None) == INV and fwd(o=None) == INV and fwd(q=258) == INV
+    assert fwd(cu=260) == INV                     # misaligned cu_seqlens
+
+    def dec(B=4, H=2, d=64, dt=binding.KDA_FP32, S=256):
+        p = lambda x: None if x is None else P(x)
+        return lib.kda_decode_step_softplus(P(256), P(256), P(256), P(256), P(256), p(S),
+                                            P(256), B, H, d, d, dt, None)
+
+    assert dec(d=48) == UNS and dec(dt=7) == UNS
+    assert dec(B=-1) == INV and dec(H=0) == INV
+    assert dec(B=0) == OK
+    assert dec(S=None) == INV and dec(S=264) == INV
