@@ -105,3 +105,52 @@ def test_packing_is_invisible(batch):
                                 np.array([0, e - s]), None if h0 is None else h0[n:n + 1])
         assert np.array_equal(o[s:e], o1)
         assert np.array_equal(hT[n:n + 1], h1)
+
+
+@SETTINGS
+@given(batches())
+def test_backward_adjoint_identity(batch):
+    """(h0, V) -> (O, hT) is linear, so its gradient is its adjoint:
+    <dO, O> + <dhT, hT> = <dh0, h0> + <dV, V> for any dO, dhT."""
+    q, k, v, g, beta, cu, h0, _ = batch
+    N, H, dk, dv = len(cu) - 1, q.shape[1], q.shape[2], v.shape[2]
+    rng = np.random.default_rng(int(cu[-1]) + 7 * N + dk)
+    h0 = rng.standard_normal((N, H, dk, dv)) if h0 is None else h0
+    d_o = rng.standard_normal(v.shape)
+    d_hT = rng.standard_normal((N, H, dk, dv))
+    o, hT = oracle.forward(q, k, v, g, beta, cu, h0)
+    gr = oracle.backward(q, k, v, g, beta, cu, h0=h0, d_o=d_o, d_hT=d_hT)
+    lhs = np.sum(d_o * o) + np.sum(d_hT * hT)
+    rhs = np.sum(gr["dh0"] * h0) + np.sum(gr["dv"] * v)
+    assert abs(lhs - rhs) <= 1e-10 * max(1.0, abs(lhs))
+
+
+@SETTINGS
+@given(batches())
+def test_backward_directional_derivative(batch):
+    """Along a random direction in every input at once, the central
+    difference of L = <dO, O> + <dhT, hT> matches the gradient's inner
+    product with the direction (finite gates, beta inside (0, 1))."""
+    q, k, v, g, beta, cu, h0, _ = batch
+    N, H, dk, dv = len(cu) - 1, q.shape[1], q.shape[2], v.shape[2]
+    g = np.clip(np.nan_to_num(g, posinf=6.0, neginf=-6.0), -6.0, 6.0)
+    beta = np.clip(beta, 0.05, 0.95)
+    rng = np.random.default_rng(int(cu[-1]) + 11 * H + dv)
+    h0 = 0.3 * rng.standard_normal((N, H, dk, dv)) if h0 is None else h0
+    d_o = rng.standard_normal(v.shape)
+    d_hT = rng.standard_normal((N, H, dk, dv))
+    x = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "h0": h0}
+    dx = {n: rng.standard_normal(a.shape) for n, a in x.items()}
+
+    def loss(eps):
+        y = {n: x[n] + eps * dx[n] for n in x}
+        o, hT = oracle.forward(y["q"], y["k"], y["v"], y["g"], y["beta"], cu, y["h0"])
+        return np.sum(d_o * o) + np.sum(d_hT * hT)
+
+    gr = oracle.backward(q, k, v, g, beta, cu, h0=h0, d_o=d_o, d_hT=d_hT)
+    names = {"q": "dq", "k": "dk", "v": "dv", "g": "dg", "beta": "dbeta", "h0": "dh0"}
+    analytic = sum(np.sum(gr[names[n]] * dx[n]) for n in x)
+    eps = 1e-5
+    numeric = (loss(eps) - loss(-eps)) / (2 * eps)
+    scale = max(1.0, abs(analytic), sum(np.sum(np.abs(gr[names[n]] * dx[n])) for n in x))
+    assert abs(numeric - analytic) <= 1e-6 * scale, (numeric, analytic)
