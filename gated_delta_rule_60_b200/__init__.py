@@ -7,6 +7,10 @@ seeded synthetic input generator.  Importing the package does not load the
 library; the first call of a binding function does, and raises if the library
 is missing.
 """
-from .binding import (KdaError, kda_chunk_fwd, kda_chunk_fwd_workspace_size,  # noqa: F401
-                      kda_decode_step, kda_status_string, kda_stream_status,
-                      kda_version, load_library)
+from .binding import (KdaError, kda_chunk_bwd, kda_chunk_bwd_workspace_size,  # noqa: F401
+                      kda_chunk_fwd, kda_chunk_fwd_gated, kda_chunk_fwd_noalloc,
+                      kda_chunk_fwd_softplus, kda_chunk_fwd_workspace_size,
+                      kda_debug_range_prefill, kda_debug_range_read,
+                      kda_debug_stall_prefill, kda_decode_step, kda_decode_step_softplus,
+                      kda_prologue, kda_selftest_wait_timeout, kda_status_string,
+                      kda_stream_status, kda_version, load_library)

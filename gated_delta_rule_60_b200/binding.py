@@ -112,6 +112,12 @@ def kda_chunk_fwd_workspace_size(N: int, T_tot: int, H: int, dk: int, dv: int,
         int(N), int(T_tot), int(H), int(dk), int(dv), _DTYPES[dtype]))
 
 
+def kda_chunk_bwd_workspace_size(N: int, T_tot: int, H: int, dk: int, dv: int,
+                                 dtype: torch.dtype) -> int:
+    return int(load_library().kda_chunk_bwd_workspace_size(
+        int(N), int(T_tot), int(H), int(dk), int(dv), _DTYPES[dtype]))
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 

@@ -271,3 +271,17 @@ def test_softplus_entry_points_checked_on_the_host(lib):
     assert dec(B=-1) == INV and dec(H=0) == INV
     assert dec(B=0) == OK
     assert dec(S=None) == INV and dec(S=264) == INV
+
+
+def test_binding_has_every_entry_point_under_its_c_name(lib):
+    """The Python binding mirrors the C ABI name for name, and the package
+    exports each of them."""
+    for name in _declared_symbols():
+        assert callable(getattr(binding, name, None)), name
+        assert getattr(kda, name) is getattr(binding, name), name
+
+
+def test_backward_workspace_query_through_the_binding(lib):
+    import torch
+    assert binding.kda_chunk_bwd_workspace_size(2, 100, 3, 64, 64, torch.float32) == \
+        lib.kda_chunk_bwd_workspace_size(2, 100, 3, 64, 64, binding.KDA_FP32) > 0
