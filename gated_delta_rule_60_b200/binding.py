@@ -7,7 +7,9 @@ operator's arithmetic runs in libkda's CUDA kernels; there is no fallback of
 any kind, and importing a function from here on a machine without the built
 library raises immediately.
 
-The Python names are the C names.
+The Python names are the C names.  As in the C ABI, the tensors of a call
+must live on the current CUDA device (select it with torch.cuda.set_device or
+a torch.cuda.device context); stream=None means that device's current stream.
 """
 import ctypes
 import os
